@@ -1,0 +1,479 @@
+/*
+ * sq_oracle.c -- plain, slow CPU oracle of the quantized-state decode step.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load this library. The product path (the
+ * CUDA library under quantized_linear_attention_sq_b200/csrc) never calls
+ * it, and the two share no code, headers, tables or helpers.
+ *
+ * What it computes (one decode step of a gated delta-rule state, kept in a
+ * low-bit, two-axis-scaled format):
+ *
+ *   - gated delta rule, per (request, value head) state S (d x d):
+ *       S <- diag(g) S ;  u = beta (v - S^T k) ;  S <- S + k u^T ;  o = S^T q
+ *     GDN has one gate per head, KDA one gate per key channel
+ *     ["STEPQuant review (e-cogni)", section "Contexto"; "STEPQuant talk
+ *     announcement (qingkeai)", opening section].
+ *   - the state is stored as S_ij ~= r_i * c_j * q_ij: a row scale per key
+ *     row, a column scale per value column, and low-bit integer codes
+ *     ["STEPQuant review (e-cogni)", "O que os autores propõem",
+ *     Key-Row-Aware Dual-Axis Fitting; talk announcement, section
+ *     "STEPQuant 核心设计"].
+ *   - bit widths are set per unit (a head for GDN, a key row for KDA) and a
+ *     few units stay in FP16 as pivots ["STEPQuant: estados recurrentes a
+ *     6 bit" (gpt-diffusion), "Las dos ideas: cuándo y dónde importa el
+ *     error"].
+ *   - after every update the state is requantized; the row scale comes from
+ *     the row's current magnitude times its calibrated row-impact factor
+ *     (same sections), so errors feed back step after step
+ *     ["STEPQuant review (e-cogni)", "Contexto"].
+ *
+ * The pages fix the method but not its arithmetic; the canonical
+ * elementwise arithmetic below is this project's reading, chosen so that
+ * two implementations agree bit for bit on the integer codes. Reductions
+ * (the two dot products per column) are the only order-free steps: here
+ * they are accumulated in fp64 from exact fp32 products and rounded once.
+ *
+ * Column-normalised form. With S = T diag(c), the whole step is carried out
+ * on T (the row-scale x code part), and c enters only where S^T k and S^T q
+ * are formed and where u is mapped back to T units:
+ *   1. a_i   = fp32(r_i * g_i)                          (quantized rows)
+ *   2. T_ij  = fp32(q_ij * a_i)        quantized rows
+ *      T_ij  = fp32(h_ij * g_i)        pivot rows (h = stored fp16 of T)
+ *   3. P_j   = sum_i T_ij k_i          (fp64 sum, rounded once to fp32)
+ *   4. p_j = fp32(c_j P_j); u_j = fp32(beta fp32(v_j - p_j));
+ *      w_j = fp32(u_j * ic_j) with ic_j = fp32(1 / c_j)
+ *   5. T'_ij = fmaf(k_i, w_j, T_ij)
+ *   6. O_j   = sum_i T'_ij q_i (fp64, rounded once); o_j = fp32(c_j O_j)
+ *   7. m_i   = max_j |T'_ij| (a NaN makes m_i NaN)
+ *   8. s_i   = fp32(fp32(phi_i m_i) / qmax_i); r'_i = fp16 of s_i rounded
+ *      toward +inf (saturating at 65504); ir_i = 0 if r'_i == 0 else
+ *      fp32(1 / r'_i)
+ *   9. q'_ij = RNE(min(max(fp32(T'_ij * ir_i), -qmax), qmax))
+ *  10. pivot rows: h'_ij = fp16 round-to-nearest-even of T'_ij, saturating
+ *      at +-65504; a NaN stores 0.
+ *  A row whose m_i is NaN stores r' = 0 and all codes 0 (status bit 0).
+ *
+ * Storage format (this project's reading; the pages give only the bit
+ * accounting): a request's state is one contiguous slot; inside it the
+ * value heads follow each other; a head's record is
+ *   [d row scales, fp16 little-endian][row 0][row 1]...[row d-1][zero pad to 16 B]
+ * A pivot row holds d fp16 values (its scale slot holds fp16 1.0). A
+ * quantized row of width b holds d codes in a little-endian bit stream:
+ * code j occupies stream bits [b*j, b*j + b), stream bit n is bit n%8 of
+ * byte n/8, and the stored field is the code plus 2^(b-1) (offset binary),
+ * so a code q in [-qmax, qmax] is stored as q + 2^(b-1) in [1, 2^b - 1].
+ * A row takes ceil(d*b/8) bytes (exactly d*b/8 for the d = 32, 64, 128 the
+ * CUDA path supports; tiny tiles used by the brute-force pins round up).
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math (oracle/build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ST_NAN 1u       /* a NaN reached the state or the output */
+#define ST_SATURATED 2u /* an fp16 value or row scale saturated at 65504 */
+#define ST_BAD_SLOT 4u  /* a slot id outside [0, n_slots) was skipped */
+
+typedef struct {
+  int32_t n_slots;
+  int32_t h_v;
+  int32_t h_k;
+  int32_t d;
+  int32_t gate_kind;         /* 0: one gate per head (GDN); 1: per key channel (KDA) */
+  const int8_t *unit_bits;   /* GDN [h_v], KDA [h_v*d]; 2, 4, 6 or 8 */
+  const uint8_t *pivot;      /* same shape; nonzero = FP16 pivot unit */
+  const float *col_scale;    /* [h_v*d] c_j */
+  const float *row_impact;   /* [h_v*d] phi_i */
+} sqo_desc;
+
+/* ------------------------------------------------------------------ fp16 */
+/* Written from the IEEE-754 binary16 definition: 1 sign bit, 5 exponent bits
+ * (bias 15), 10 fraction bits; subnormals have quantum 2^-24. */
+
+float sqo_f16_to_f32(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0)
+    v = ldexp((double)m, -24);
+  else if (e == 31)
+    v = m ? NAN : INFINITY;
+  else
+    v = ldexp((double)(m | 0x400), e - 25);
+  return (float)(sign ? -v : v);
+}
+
+/* Encode |value| = n * 2^qexp (n integer, 0 <= n <= 2048) as fp16 bits. */
+static uint16_t f16_encode(int sign, double n, int qexp) {
+  uint16_t s = sign ? 0x8000 : 0;
+  if (n == 0.0) return s;
+  if (n >= 2048.0) { n = 1024.0; qexp += 1; }
+  if (n < 1024.0) return (uint16_t)(s | (uint16_t)n); /* subnormal, qexp == -24 */
+  int ef = qexp + 25;
+  if (ef >= 31) return (uint16_t)(s | 0x7c00);
+  return (uint16_t)(s | (ef << 10) | ((int)n - 1024));
+}
+
+/* The quantum (spacing) of fp16 numbers around a finite a >= 0, as 2^qexp. */
+static int f16_quantum_exp(double a) {
+  if (a < ldexp(1.0, -14)) return -24;
+  int e;
+  frexp(a, &e); /* a = f 2^e, f in [0.5, 1) */
+  return e - 11;
+}
+
+/* round to nearest, ties to even */
+uint16_t sqo_f16_rne(float x) {
+  if (isnan(x)) return 0x7e00;
+  int sign = signbit(x) ? 1 : 0;
+  double a = fabs((double)x);
+  if (isinf(x) || a >= 65520.0) return (uint16_t)(sign ? 0xfc00 : 0x7c00);
+  int qe = f16_quantum_exp(a);
+  double n = nearbyint(ldexp(a, -qe)); /* default rounding mode: nearest-even */
+  return f16_encode(sign, n, qe);
+}
+
+/* round toward +infinity */
+uint16_t sqo_f16_ru(float x) {
+  if (isnan(x)) return 0x7e00;
+  int sign = signbit(x) ? 1 : 0;
+  double a = fabs((double)x);
+  if (isinf(x)) return (uint16_t)(sign ? 0xfbff : 0x7c00);
+  if (!sign && a > 65504.0) return 0x7c00;
+  if (sign && a > 65504.0) return 0xfbff;
+  int qe = f16_quantum_exp(a);
+  double t = ldexp(a, -qe);
+  double n = sign ? floor(t) : ceil(t); /* toward +inf: down in magnitude for negatives */
+  return f16_encode(sign, n, qe);
+}
+
+/* -------------------------------------------------------------- layout */
+
+static int unit_index(const sqo_desc *D, int h, int i) {
+  return D->gate_kind == 0 ? h : h * D->d + i;
+}
+static int row_is_pivot(const sqo_desc *D, int h, int i) {
+  return D->pivot[unit_index(D, h, i)] != 0;
+}
+static int row_width(const sqo_desc *D, int h, int i) {
+  return D->unit_bits[unit_index(D, h, i)];
+}
+static size_t row_bytes(const sqo_desc *D, int h, int i) {
+  if (row_is_pivot(D, h, i)) return (size_t)2 * D->d;
+  return ((size_t)D->d * (size_t)row_width(D, h, i) + 7) / 8;
+}
+size_t sqo_record_bytes(const sqo_desc *D, int h) {
+  size_t n = (size_t)2 * D->d;
+  for (int i = 0; i < D->d; i++) n += row_bytes(D, h, i);
+  return (n + 15) / 16 * 16;
+}
+size_t sqo_slot_bytes(const sqo_desc *D) {
+  size_t n = 0;
+  for (int h = 0; h < D->h_v; h++) n += sqo_record_bytes(D, h);
+  return n;
+}
+size_t sqo_head_offset(const sqo_desc *D, int h) {
+  size_t n = 0;
+  for (int hh = 0; hh < h; hh++) n += sqo_record_bytes(D, hh);
+  return n;
+}
+size_t sqo_pool_bytes(const sqo_desc *D) { return sqo_slot_bytes(D) * (size_t)D->n_slots; }
+
+static size_t row_offset(const sqo_desc *D, int h, int i) {
+  size_t n = (size_t)2 * D->d;
+  for (int ii = 0; ii < i; ii++) n += row_bytes(D, h, ii);
+  return n;
+}
+
+/* ------------------------------------------------------- bit streams */
+
+static void put_bit(uint8_t *p, long n, unsigned bit) {
+  uint8_t mask = (uint8_t)(1u << (n % 8));
+  if (bit) p[n / 8] |= mask; else p[n / 8] &= (uint8_t)~mask;
+}
+static unsigned get_bit(const uint8_t *p, long n) { return (p[n / 8] >> (n % 8)) & 1u; }
+
+/* store code q (in [-qmax, qmax]) as field q + 2^(b-1) at position j */
+void sqo_put_code(uint8_t *row, int b, int j, int q) {
+  unsigned field = (unsigned)(q + (1 << (b - 1)));
+  for (int t = 0; t < b; t++) put_bit(row, (long)b * j + t, (field >> t) & 1u);
+}
+int sqo_get_code(const uint8_t *row, int b, int j) {
+  unsigned field = 0;
+  for (int t = 0; t < b; t++) field |= get_bit(row, (long)b * j + t) << t;
+  return (int)field - (1 << (b - 1));
+}
+
+static uint16_t rd16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static void wr16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)(v & 0xff); p[1] = (uint8_t)(v >> 8); }
+
+static int qmax_of(int b) { return (1 << (b - 1)) - 1; }
+
+/* ------------------------------------------------ per-tile primitives */
+
+/* Read a head record into column-normalised T (d x d), applying the
+ * per-row multiplier: a_i = r_i * g_i for quantized rows, g_i for pivots.
+ * With gate == NULL the multiplier is r_i (quantized) and 1 (pivots), and no
+ * rounding beyond the exact q * r product happens. */
+static void load_T(const sqo_desc *D, int h, const uint8_t *rec, const float *gate, float *T) {
+  int d = D->d;
+  for (int i = 0; i < d; i++) {
+    const uint8_t *row = rec + row_offset(D, h, i);
+    if (row_is_pivot(D, h, i)) {
+      for (int j = 0; j < d; j++) {
+        float hv = sqo_f16_to_f32(rd16(row + 2 * j));
+        T[i * d + j] = gate ? hv * gate[i] : hv;
+      }
+    } else {
+      int b = row_width(D, h, i);
+      float r = sqo_f16_to_f32(rd16(rec + 2 * i));
+      float a = gate ? r * gate[i] : r;
+      for (int j = 0; j < d; j++) T[i * d + j] = (float)sqo_get_code(row, b, j) * a;
+    }
+  }
+}
+
+/* Steps 7-10: requantize column-normalised T' into the record. */
+static uint32_t store_T(const sqo_desc *D, int h, uint8_t *rec, const float *T) {
+  int d = D->d;
+  uint32_t st = 0;
+  const float *phi = D->row_impact + (size_t)h * d;
+  memset(rec, 0, sqo_record_bytes(D, h));
+  for (int i = 0; i < d; i++) {
+    uint8_t *row = rec + row_offset(D, h, i);
+    const float *t = T + (size_t)i * d;
+    if (row_is_pivot(D, h, i)) {
+      wr16(rec + 2 * i, 0x3c00);
+      for (int j = 0; j < d; j++) {
+        float x = t[j];
+        uint16_t hv;
+        if (isnan(x)) { hv = 0; st |= ST_NAN; }
+        else if (fabsf(x) > 65504.0f) { hv = signbit(x) ? 0xfbff : 0x7bff; st |= ST_SATURATED; }
+        else hv = sqo_f16_rne(x);
+        wr16(row + 2 * j, hv);
+      }
+      continue;
+    }
+    int b = row_width(D, h, i);
+    int qm = qmax_of(b);
+    /* 7. row magnitude */
+    float m = 0.0f;
+    int has_nan = 0;
+    for (int j = 0; j < d; j++) {
+      if (isnan(t[j])) has_nan = 1;
+      else if (fabsf(t[j]) > m) m = fabsf(t[j]);
+    }
+    if (has_nan) {
+      st |= ST_NAN;
+      wr16(rec + 2 * i, 0);
+      for (int j = 0; j < d; j++) sqo_put_code(row, b, j, 0);
+      continue;
+    }
+    /* 8. row scale from magnitude x row impact, rounded up to fp16 */
+    float s = (phi[i] * m) / (float)qm;
+    uint16_t rb;
+    if (s > 65504.0f) { rb = 0x7bff; st |= ST_SATURATED; }
+    else rb = sqo_f16_ru(s);
+    wr16(rec + 2 * i, rb);
+    float r = sqo_f16_to_f32(rb);
+    float ir = (r == 0.0f) ? 0.0f : 1.0f / r;
+    /* 9. codes: round half to even after clamping to the symmetric range */
+    for (int j = 0; j < d; j++) {
+      float y = t[j] * ir;
+      if (y > (float)qm) y = (float)qm;
+      if (y < -(float)qm) y = -(float)qm;
+      sqo_put_code(row, b, j, (int)nearbyintf(y));
+    }
+  }
+  return st;
+}
+
+static const float *gate_vector(const sqo_desc *D, const float *g, int b, int h, float *buf) {
+  int d = D->d;
+  if (D->gate_kind == 0) {
+    for (int i = 0; i < d; i++) buf[i] = g[(size_t)b * D->h_v + h];
+    return buf;
+  }
+  return g + ((size_t)b * D->h_v + h) * d;
+}
+
+static int slot_of(const sqo_desc *D, const int32_t *slots, int b, uint32_t *st) {
+  int s = slots ? slots[b] : b;
+  if (s < 0 || s >= D->n_slots) { *st |= ST_BAD_SLOT; return -1; }
+  return s;
+}
+
+/* One quantized-format decode step for one (request b, value head h) tile. */
+static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
+                          const float *q_all, const float *k_all, const float *v_all,
+                          const float *beta_all, const float *g_all, float *o_all,
+                          float *T, float *gbuf, float *w) {
+  int d = D->d;
+  int hk = h / (D->h_v / D->h_k);
+  const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
+  const float *k = k_all + ((size_t)b * D->h_k + hk) * d;
+  const float *v = v_all + ((size_t)b * D->h_v + h) * d;
+  float beta = beta_all[(size_t)b * D->h_v + h];
+  float *o = o_all + ((size_t)b * D->h_v + h) * d;
+  const float *c = D->col_scale + (size_t)h * d;
+  const float *gate = gate_vector(D, g_all, b, h, gbuf);
+  uint32_t st = 0;
+
+  load_T(D, h, rec, gate, T);                          /* steps 1-2 */
+  for (int j = 0; j < d; j++) {                        /* steps 3-4 */
+    double acc = 0.0;
+    for (int i = 0; i < d; i++) acc += (double)T[i * d + j] * (double)k[i];
+    float P = (float)acc;
+    float p = c[j] * P;
+    float u = beta * (v[j] - p);
+    float ic = 1.0f / c[j];
+    w[j] = u * ic;
+  }
+  for (int i = 0; i < d; i++)                          /* step 5 */
+    for (int j = 0; j < d; j++) T[i * d + j] = fmaf(k[i], w[j], T[i * d + j]);
+  for (int j = 0; j < d; j++) {                        /* step 6 */
+    double acc = 0.0;
+    for (int i = 0; i < d; i++) acc += (double)T[i * d + j] * (double)q[i];
+    float O = (float)acc;
+    o[j] = c[j] * O;
+    if (isnan(o[j])) st |= ST_NAN;
+  }
+  st |= store_T(D, h, rec, T);                         /* steps 7-10 */
+  return st;
+}
+
+/* ------------------------------------------------------ public entry */
+
+/* One decode step for batch rows [b0, b1) of a quantized pool. Inputs:
+ * q, k [B, h_k, d]; v [B, h_v, d]; beta [B, h_v]; g [B, h_v] (GDN) or
+ * [B, h_v, d] (KDA); o [B, h_v, d]; slots [B] or NULL (identity). Returns
+ * the status bits. Tiles of a skipped slot write o = 0. */
+uint32_t sqo_step_range(const sqo_desc *D, uint8_t *pool, const float *q, const float *k,
+                        const float *v, const float *beta, const float *g, float *o,
+                        const int32_t *slots, int b0, int b1) {
+  int d = D->d;
+  float *T = malloc(sizeof(float) * d * d);
+  float *gbuf = malloc(sizeof(float) * d);
+  float *w = malloc(sizeof(float) * d);
+  uint32_t st = 0;
+  size_t slot_bytes = sqo_slot_bytes(D);
+  for (int b = b0; b < b1; b++) {
+    int s = slot_of(D, slots, b, &st);
+    for (int h = 0; h < D->h_v; h++) {
+      if (s < 0) {
+        memset(o + ((size_t)b * D->h_v + h) * d, 0, sizeof(float) * d);
+        continue;
+      }
+      uint8_t *rec = pool + (size_t)s * slot_bytes + sqo_head_offset(D, h);
+      st |= step_tile(D, rec, b, h, q, k, v, beta, g, o, T, gbuf, w);
+    }
+  }
+  free(T); free(gbuf); free(w);
+  return st;
+}
+
+uint32_t sqo_step(const sqo_desc *D, uint8_t *pool, const float *q, const float *k,
+                  const float *v, const float *beta, const float *g, float *o,
+                  const int32_t *slots, int B) {
+  return sqo_step_range(D, pool, q, k, v, beta, g, o, slots, 0, B);
+}
+
+/* Quantize fp32 states S [B, h_v, d, d] (S-space) into the pool slots:
+ * T_ij = fp32(S_ij * ic_j), then steps 7-10. */
+uint32_t sqo_quantize(const sqo_desc *D, uint8_t *pool, const float *S, const int32_t *slots, int B) {
+  int d = D->d;
+  float *T = malloc(sizeof(float) * d * d);
+  uint32_t st = 0;
+  size_t slot_bytes = sqo_slot_bytes(D);
+  for (int b = 0; b < B; b++) {
+    int s = slot_of(D, slots, b, &st);
+    if (s < 0) continue;
+    for (int h = 0; h < D->h_v; h++) {
+      const float *Sh = S + ((size_t)b * D->h_v + h) * d * d;
+      const float *c = D->col_scale + (size_t)h * d;
+      for (int i = 0; i < d; i++)
+        for (int j = 0; j < d; j++) {
+          float ic = 1.0f / c[j];
+          T[i * d + j] = Sh[i * d + j] * ic;
+        }
+      st |= store_T(D, h, pool + (size_t)s * slot_bytes + sqo_head_offset(D, h), T);
+    }
+  }
+  free(T);
+  return st;
+}
+
+/* Dequantize pool slots into S [B, h_v, d, d]: S_ij = fp32(fp32(q r) c_j)
+ * for quantized rows and fp32(h c_j) for pivot rows. Skipped slots give 0. */
+uint32_t sqo_dequantize(const sqo_desc *D, const uint8_t *pool, float *S, const int32_t *slots, int B) {
+  int d = D->d;
+  float *T = malloc(sizeof(float) * d * d);
+  uint32_t st = 0;
+  size_t slot_bytes = sqo_slot_bytes(D);
+  for (int b = 0; b < B; b++) {
+    int s = slot_of(D, slots, b, &st);
+    for (int h = 0; h < D->h_v; h++) {
+      float *Sh = S + ((size_t)b * D->h_v + h) * d * d;
+      if (s < 0) { memset(Sh, 0, sizeof(float) * d * d); continue; }
+      const float *c = D->col_scale + (size_t)h * d;
+      load_T(D, h, pool + (size_t)s * slot_bytes + sqo_head_offset(D, h), NULL, T);
+      for (int i = 0; i < d; i++)
+        for (int j = 0; j < d; j++) Sh[i * d + j] = T[i * d + j] * c[j];
+    }
+  }
+  free(T);
+  return st;
+}
+
+/* Unquantized FP32 state step (S-space), S pool [n_slots, h_v, d, d]:
+ *   G = g_i S_ij ; P_j = sum_i G_ij k_i ; u_j = beta (v_j - P_j) ;
+ *   S'_ij = fmaf(k_i, u_j, G_ij) ; o_j = sum_i S'_ij q_i. */
+uint32_t sqo_step_fp32_range(const sqo_desc *D, float *Spool, const float *q_all, const float *k_all,
+                             const float *v_all, const float *beta_all, const float *g_all, float *o_all,
+                             const int32_t *slots, int b0, int b1) {
+  int d = D->d;
+  float *gbuf = malloc(sizeof(float) * d);
+  float *u = malloc(sizeof(float) * d);
+  uint32_t st = 0;
+  for (int b = b0; b < b1; b++) {
+    int s = slot_of(D, slots, b, &st);
+    for (int h = 0; h < D->h_v; h++) {
+      float *o = o_all + ((size_t)b * D->h_v + h) * d;
+      if (s < 0) { memset(o, 0, sizeof(float) * d); continue; }
+      int hk = h / (D->h_v / D->h_k);
+      const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
+      const float *k = k_all + ((size_t)b * D->h_k + hk) * d;
+      const float *v = v_all + ((size_t)b * D->h_v + h) * d;
+      float beta = beta_all[(size_t)b * D->h_v + h];
+      const float *gate = gate_vector(D, g_all, b, h, gbuf);
+      float *S = Spool + ((size_t)s * D->h_v + h) * d * d;
+      for (int i = 0; i < d; i++)
+        for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
+      for (int j = 0; j < d; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)k[i];
+        float P = (float)acc;
+        u[j] = beta * (v[j] - P);
+      }
+      for (int i = 0; i < d; i++)
+        for (int j = 0; j < d; j++) S[i * d + j] = fmaf(k[i], u[j], S[i * d + j]);
+      for (int j = 0; j < d; j++) {
+        double acc = 0.0;
+        for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)q[i];
+        o[j] = (float)acc;
+        if (isnan(o[j])) st |= ST_NAN;
+      }
+    }
+  }
+  free(gbuf); free(u);
+  return st;
+}
+
+uint32_t sqo_step_fp32(const sqo_desc *D, float *Spool, const float *q, const float *k, const float *v,
+                       const float *beta, const float *g, float *o, const int32_t *slots, int B) {
+  return sqo_step_fp32_range(D, Spool, q, k, v, beta, g, o, slots, 0, B);
+}
