@@ -1,0 +1,333 @@
+"""Benchmark of the quantized-state decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: GDN serving scale -- batch 512 requests x 32 value heads (16 key
+heads), d = 128, 6-bit nominal budget with per-head widths {4, 6, 8} and 5 %
+FP16 pivot heads, state warmed up by 64 unquantized steps with 2 % outlier
+columns x20 (synthetic, seeded). One step = one decode step of every
+(request, head) state tile = one launch of the fused kernel.
+
+Prints one JSON line (rank 0). ``value`` is (request*head)-steps/s over all
+ranks with inputs resident in HBM; ``e2e`` is the same through the public
+API with the step's activations copied from pinned host memory and o copied
+back inside the timed region; ``roofline`` compares the kernel's algorithmic
+state bytes (codes + row scales + pivots, read and written once) per launch
+with the measured HBM copy bandwidth; ``cpu_baseline`` times the CPU oracle
+on a bounded sample of the same workload.
+
+Multi-GPU: each rank owns its own 512 requests (requests are independent;
+no collective on the data path) -> weak scaling; timing is the max over
+ranks. ``--impl reference`` times the CPU oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-state decode (request·head)-steps/s; achieved HBM GB/s vs B200 peak"
+UNIT = "(request*head)-steps/s"
+CONFIG_ID = 3
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(w):
+    c = w.cfg
+    return {"workload": c.name, "batch_per_gpu": c.batch, "h_v": c.h_v, "h_k": c.h_k, "d": c.d,
+            "gate": "GDN (one gate per head)", "widths": "per-head {4,6,8}, 6-bit nominal, 5% FP16 pivot heads",
+            "warmup": f"{c.warmup_steps} unquantized steps, 2% outlier columns x20",
+            "l2": "state 222 MB > 126 MB L2 (no flush); 8 rotating input sets"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from quantized_linear_attention_sq_b200 import _abi, build, synth
+    from quantized_linear_attention_sq_b200.state import StatePool
+
+    torch.cuda.set_device(local_rank)
+    build.build()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = synth.workload(CONFIG_ID, seed=args.seed + rank)   # each rank: its own 512 requests
+    c = w.cfg
+    cal = w.calib()
+    B = c.batch
+    dev = torch.device("cuda", local_rank)
+
+    def make(fmt):
+        return StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, fmt, cal.unit_bits, cal.pivot, cal.col_scale,
+                         cal.row_impact)
+
+    # initial state: S0, 64 unquantized warm-up steps on the GPU (FP32 kernel), outliers, quantize
+    S = torch.from_numpy(w.initial_state()).to(dev)
+    fp = make(_abi.SQ_FMT_FP32)
+    o = torch.empty((B, c.h_v, c.d), device=dev)
+    for t in range(-c.warmup_steps, 0):
+        q, k, v, beta, g = (torch.from_numpy(x).to(dev) for x in w.step_inputs(t))
+        fp.decode_step(S, q, k, v, beta, g, o)
+    S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
+    sp = make(_abi.SQ_FMT_PACKED)
+    pool = sp.new_pool()
+    sp.quantize_state(pool, S)
+    torch.cuda.synchronize()
+    NI = 8
+    host_inputs = [w.step_inputs(t) for t in range(NI)]
+    dev_inputs = [[torch.from_numpy(x).to(dev) for x in xs] for xs in host_inputs]
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-resident timing (per-launch events on the launching stream)
+    def timed_device(spool, pl, K, W):
+        for i in range(W):
+            spool.decode_step(pl, *dev_inputs[i % NI], o)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        n0 = spool.launches()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            spool.decode_step(pl, *dev_inputs[i % NI], o)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        launches = spool.launches() - n0
+        per = [a.elapsed_time(b) for a, b in ev]
+        return t0.elapsed_time(t1), per, launches
+
+    props = torch.cuda.get_device_properties(local_rank)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
+    with ClockSampler(gpu_id) as clk:
+        total_ms, per_ms, launches = timed_device(sp, pool, args.steps, args.warmup)
+    clocks = clk.summary()
+    total_ms = max_over_ranks(total_ms)
+    kern_ms = statistics.mean(per_ms)
+    # ---- end to end through the public API: pinned host activations in, o out
+    pinned = [[torch.from_numpy(x).pin_memory() for x in xs] for xs in host_inputs]
+    o_host = torch.empty((B, c.h_v, c.d), dtype=torch.float32).pin_memory()
+    staging = [torch.empty_like(x) for x in dev_inputs[0]]
+    h2d = sum(x.numel() * x.element_size() for x in pinned[0])
+    d2h = o_host.numel() * o_host.element_size()
+    for i in range(args.warmup):
+        for dst, src in zip(staging, pinned[i % NI]):
+            dst.copy_(src, non_blocking=True)
+        sp.decode_step(pool, *staging, o)
+        o_host.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        for dst, src in zip(staging, pinned[i % NI]):
+            dst.copy_(src, non_blocking=True)
+        sp.decode_step(pool, *staging, o)
+        o_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    st_bits = sp.get_status()
+    # ---- FP32-state step on the same workload (unquantized comparison)
+    fp_pool = S  # warmed-up fp32 state, same requests
+    fp_total, fp_per, _ = timed_device(fp, fp_pool, max(4, args.steps // 4), args.warmup)
+    fp_total = max_over_ranks(fp_total)
+    rep = sp.report
+    frep = fp.report
+    units = B * c.h_v
+    value = world * units * args.steps / (total_ms / 1e3)
+    bytes_launch = B * rep["state_bytes_per_step"]
+    peak, peak_kind = peaks()
+    achieved = bytes_launch / (kern_ms / 1e3) / 1e9
+    fp_bytes = B * frep["state_bytes_per_step"]
+    fp_kern = statistics.mean(fp_per)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
+        "config": workload_config(w),
+        "e2e": {"value": world * units * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "k_decode_step<128,packed>", "algorithmic_bytes_per_launch": bytes_launch,
+                     "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+        "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
+                  "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_bits": st_bits},
+        "fp32_state": {"value": world * units * max(4, args.steps // 4) / (fp_total / 1e3),
+                       "kernel_ms": fp_kern, "achieved_gbs": fp_bytes / (fp_kern / 1e3) / 1e9,
+                       "frac": fp_bytes / (fp_kern / 1e3) / 1e9 / peak,
+                       "speedup_quantized_vs_fp32": fp_kern / kern_ms},
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args, sample_requests=args.cpu_sample_requests)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    sp.close()
+    fp.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------- the CPU oracle
+def cpu_baseline(args, sample_requests=64, steps=None):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload:
+    `sample_requests` requests x 32 heads, `steps` decode steps, tiles split
+    over all host cores."""
+    import oracle
+    from quantized_linear_attention_sq_b200 import synth
+
+    w = synth.workload(CONFIG_ID, seed=args.seed)
+    c = w.cfg
+    cal = w.calib()
+    reqs = list(range(sample_requests))
+    o_ = oracle.Oracle(len(reqs), c.h_v, c.h_k, c.d, c.gate_kind, cal.unit_bits, cal.pivot, cal.col_scale,
+                       cal.row_impact)
+    pool = o_.new_pool()
+    S = w.initial_state(reqs)
+    S *= w.outlier_mask()[None, :, None, :]
+    o_.quantize(pool, S)
+    cores = oracle.cores_available()
+    steps = steps or args.cpu_steps
+    inputs = [w.step_inputs(t, reqs) for t in range(steps)]
+    t0 = time.perf_counter()
+    for t in range(steps):
+        o_.step(pool, *inputs[t], threads=cores)
+    dt = time.perf_counter() - t0
+    units = len(reqs) * c.h_v * steps
+    return {"value": units / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(reqs)} of {c.batch} requests x {c.h_v} heads x {steps} steps "
+                      f"({units} tile-steps, {dt:.1f} s wall on {cores} threads)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    cb = cpu_baseline(args, sample_requests=args.cpu_sample_requests, steps=max(1, args.steps))
+    from quantized_linear_attention_sq_b200 import synth
+    w = synth.workload(CONFIG_ID, seed=args.seed)
+    out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
+           "config": workload_config(w), "cpu_baseline": cb,
+           "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "note": "reference arm = the plain CPU oracle of the same step (no upstream code exists to install)"}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-requests", type=int, default=48)
+    ap.add_argument("--cpu-steps", type=int, default=4)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

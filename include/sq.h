@@ -1,0 +1,176 @@
+/*
+ * sq.h -- C ABI of the quantized recurrent-state decode step for gated
+ * delta-rule linear attention (GDN: one gate per head; KDA: one gate per key
+ * channel), B200 (sm_100a).
+ *
+ * The method (STEPQuant): every request keeps, per value head, a d x d state
+ * S (row i = key channel, column j = value channel) that a decode step
+ * updates with the gated delta rule
+ *     S <- diag(g) S ;  u = beta (v - S^T k) ;  S <- S + k u^T ;  o = S^T q
+ * ("STEPQuant review (e-cogni)", section "Contexto"; "STEPQuant talk
+ * announcement (qingkeai)", opening section). Between steps the state lives
+ * in a compressed form, S_ij ~= r_i c_j q_ij, with a row scale per key row
+ * taken from the row's current magnitude and its calibrated row-impact
+ * factor, a calibrated column scale per value column, and low-bit codes
+ * whose width is set per unit (a head for GDN, a key row for KDA); a few
+ * units are kept as FP16 pivots ("STEPQuant review (e-cogni)", section
+ * "O que os autores propõem"; "STEPQuant: estados recurrentes a 6 bit"
+ * (gpt-diffusion), section "Las dos ideas: cuándo y dónde importa el
+ * error"). Each step reads that state once, updates it in FP32, and
+ * requantizes it in place ("STEPQuant: estados recurrentes a 6 bit",
+ * "Las dos ideas", fused kernels on packed states).
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" are CUDA device pointers on the device that was
+ *    current when the handle was created; they must be 16-byte aligned and
+ *    the arrays C-contiguous. Pointers named "host" are host memory.
+ *  - Every call that takes a stream is asynchronous on that stream
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream),
+ *    except sq_get_status, which synchronizes it.
+ *  - Invalid arguments are rejected on the host with SQ_ERR_INVALID_ARG and
+ *    nothing is launched; sq_last_error() then returns a message.
+ *  - Bad data found on the device (NaN, fp16 overflow, a slot id out of
+ *    range) never traps: the kernel writes defined values and ORs a bit into
+ *    the handle's device status word (SQ_STATUS_*), read by sq_get_status.
+ *  - There is no CPU fallback: without a usable CUDA device every call that
+ *    launches work returns SQ_ERR_CUDA.
+ *  - Calls on one handle from different host threads must be serialized by
+ *    the caller. Two steps in flight on the same pool slots race.
+ *
+ * Storage format (SQ_FMT_PACKED). The pool is caller-owned device memory of
+ * sq_state_bytes().pool_bytes bytes. Slot s starts at s * slot_bytes; in it
+ * the value heads follow each other (sq_head_layout gives each head's
+ * offset and record size). A head record is
+ *     [d row scales r_i, fp16 LE][row 0][row 1] ... [row d-1][zero pad to 16 B]
+ * A pivot row is d fp16 values of the column-normalised state T = S / c
+ * (its scale slot holds fp16 1.0). A quantized row of width b in {2,4,6,8}
+ * is a little-endian bit stream of d fields of b bits: field j holds
+ * q_ij + 2^(b-1) (offset binary), q_ij in [-(2^(b-1)-1), 2^(b-1)-1].
+ * SQ_FMT_FP32 pools are plain fp32 S [n_slots][h_v][d][d].
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1,  /* rejected on the host; nothing launched */
+  SQ_ERR_UNSUPPORTED = 2,  /* valid but not built (e.g. d not in {32, 64, 128}) */
+  SQ_ERR_CUDA = 3,         /* a CUDA runtime call failed; see sq_last_error() */
+  SQ_ERR_OOM = 4           /* device allocation of the handle's tables failed */
+} sq_status;
+
+typedef enum { SQ_FMT_FP32 = 0, SQ_FMT_PACKED = 1 } sq_format;
+typedef enum { SQ_GATE_HEAD = 0 /* GDN */, SQ_GATE_KEY_CHANNEL = 1 /* KDA */ } sq_gate_kind;
+
+/* Bits of the device status word. */
+#define SQ_STATUS_NAN 1u        /* a NaN reached the updated state or o */
+#define SQ_STATUS_SATURATED 2u  /* a row scale or pivot value saturated at +-65504 */
+#define SQ_STATUS_BAD_SLOT 4u   /* a slot id outside [0, n_slots) was skipped (o = 0) */
+#define SQ_STATUS_TIMEOUT 8u    /* a bounded device wait gave up (should never happen) */
+
+/* Shape of one layer's state pool. d_k == d_v == d, d in {32, 64, 128};
+ * h_v % h_k == 0 (value head h reads key head h / (h_v / h_k)). */
+typedef struct {
+  int32_t n_slots;   /* requests the pool can hold */
+  int32_t h_v;       /* value heads (states per request) */
+  int32_t h_k;       /* key heads */
+  int32_t d_k;
+  int32_t d_v;
+  int32_t fmt;       /* sq_format */
+  int32_t gate;      /* sq_gate_kind */
+} sq_state_desc;
+
+/* Calibration tables, host memory, copied by sq_state_alloc (the caller
+ * keeps ownership). Units are heads (GATE_HEAD) or key rows (GATE_KEY_CHANNEL).
+ * Ignored (may be NULL) for SQ_FMT_FP32. */
+typedef struct {
+  const int8_t* unit_bits;    /* [h_v] or [h_v*d_k]; 2, 4, 6 or 8 */
+  const uint8_t* pivot_mask;  /* same shape; nonzero = FP16 pivot unit (overrides unit_bits) */
+  const float* col_scale;     /* [h_v*d_v] c_j, finite and > 0 */
+  const float* row_impact;    /* [h_v*d_k] phi_i, finite and > 0 */
+} sq_calib;
+
+typedef struct sq_handle sq_handle;
+
+typedef struct {
+  uint64_t pool_bytes;             /* n_slots * slot_bytes */
+  uint64_t slot_bytes;             /* one request's state, all heads */
+  uint64_t state_bytes_per_step;   /* per request: slot read + slot written by one step */
+  uint64_t act_bytes_per_step;     /* per request: q, k, v, beta, g read and o written */
+  double bits_per_value;           /* 8 * slot_bytes / (h_v * d_k * d_v) */
+  uint64_t max_record_bytes;       /* largest head record */
+} sq_bytes_report;
+
+/* Create a handle: validate the description and calibration, build the
+ * record layout and upload the per-head tables (ic_j = 1/c_j included) to
+ * the current device with cudaMalloc + cudaMemcpyAsync on `stream`. The
+ * state pool itself is NOT allocated: the caller allocates pool_bytes
+ * (returned in *pool_bytes) of device memory. Returns SQ_ERR_INVALID_ARG for
+ * bad shapes or tables, SQ_ERR_UNSUPPORTED for d not in {32, 64, 128},
+ * SQ_ERR_OOM if the tables cannot be allocated. */
+sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void* stream,
+                         sq_handle** out, size_t* pool_bytes);
+
+/* Release the handle's device tables (synchronizes the device first). NULL is a no-op. */
+sq_status sq_state_free(sq_handle* h);
+
+/* Quantize B fp32 states into pool slots ("STEPQuant review (e-cogni)",
+ * "O que os autores propõem", dual-axis fitting: T = S / c, row scales from
+ * the current row magnitude times phi, codes rounded to nearest even).
+ *   S        device fp32 [B, h_v, d, d], S-space (row = key channel)
+ *   slot_ids device int32 [B], or NULL for slots 0..B-1
+ * B == 0 is a no-op. FP32 pools: a plain copy. */
+sq_status sq_quantize_state(sq_handle* h, void* pool, const float* S, const int32_t* slot_ids,
+                            int32_t B, void* stream);
+
+/* One decode step for B requests, in place on the pool ("STEPQuant review
+ * (e-cogni)", "Contexto": gated delta rule; talk announcement, "STEPQuant
+ * 核心设计": row scales from magnitude and impact, column scales; gpt-diffusion
+ * page, "Las dos ideas": fused kernels on packed states):
+ *   q, k     device fp32 [B, h_k, d]
+ *   v        device fp32 [B, h_v, d]
+ *   beta     device fp32 [B, h_v]
+ *   g        device fp32 [B, h_v] (GATE_HEAD) or [B, h_v, d] (GATE_KEY_CHANNEL)
+ *   o        device fp32 [B, h_v, d], written: o = S'^T q from the updated
+ *            state before requantization
+ *   slot_ids device int32 [B] (distinct), or NULL for slots 0..B-1
+ * Reads and writes each touched state record exactly once. */
+sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* k, const float* v,
+                         const float* beta, const float* g, float* o, const int32_t* slot_ids,
+                         int32_t B, void* stream);
+
+/* Expand B pool slots to fp32 S [B, h_v, d, d] (device): S_ij = (q r) c_j for
+ * quantized rows and h c_j for pivot rows. Skipped (bad) slots give 0. */
+sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, const int32_t* slot_ids,
+                              int32_t B, void* stream);
+
+/* Byte accounting of the layout (host only, no device work). */
+sq_status sq_state_bytes(const sq_handle* h, sq_bytes_report* out);
+
+/* Offset within a slot and size of value head `head`'s record (host only). */
+sq_status sq_head_layout(const sq_handle* h, int32_t head, uint64_t* offset, uint64_t* record_bytes);
+
+/* Synchronize `stream`, return the device status bits accumulated since the
+ * last clear, and clear them if `clear` is nonzero. */
+sq_status sq_get_status(sq_handle* h, void* stream, uint32_t* bits, int32_t clear);
+
+/* Number of kernel launches this handle has issued (host-side counter). */
+uint64_t sq_launch_count(const sq_handle* h);
+
+/* Message for the last non-OK return on this host thread ("" if none). */
+const char* sq_last_error(void);
+
+/* Library version string. */
+const char* sq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_H */

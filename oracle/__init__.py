@@ -20,6 +20,7 @@ from __future__ import annotations
 import ctypes
 import os
 import threading
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
 import numpy as np
@@ -57,10 +58,10 @@ def lib():
             for f in ("sqo_slot_bytes", "sqo_pool_bytes"):
                 getattr(L, f).argtypes = [P]
                 getattr(L, f).restype = ctypes.c_size_t
-            L.sqo_step_range.argtypes = [P] * 9 + [ctypes.c_int, ctypes.c_int]
-            L.sqo_step_range.restype = ctypes.c_uint32
-            L.sqo_step_fp32_range.argtypes = [P] * 9 + [ctypes.c_int, ctypes.c_int]
-            L.sqo_step_fp32_range.restype = ctypes.c_uint32
+            L.sqo_step_tiles.argtypes = [P] * 9 + [ctypes.c_int, ctypes.c_int]
+            L.sqo_step_tiles.restype = ctypes.c_uint32
+            L.sqo_step_fp32_tiles.argtypes = [P] * 9 + [ctypes.c_int, ctypes.c_int]
+            L.sqo_step_fp32_tiles.restype = ctypes.c_uint32
             L.sqo_quantize.argtypes = [P, P, P, P, ctypes.c_int]
             L.sqo_quantize.restype = ctypes.c_uint32
             L.sqo_dequantize.argtypes = [P, P, P, P, ctypes.c_int]
@@ -136,30 +137,35 @@ class Oracle:
         st = lib().sqo_dequantize(self._dp, _ptr(pool), _ptr(S), _ptr(slots), B)
         return S, st
 
-    def step(self, pool, q, k, v, beta, g, slots=None, b0=0, b1=None, o=None):
-        """Quantized decode step in place on ``pool``; returns (o, status)."""
+    def _run_tiles(self, fn, state, q, k, v, beta, g, slots, o, threads, tiles):
         q, k, v, beta, g = (_c(x, np.float32) for x in (q, k, v, beta, g))
         slots = _c(slots, np.int32)
         B = q.shape[0]
         if o is None:
             o = np.zeros((B, self.h_v, self.d), dtype=np.float32)
-        b1 = B if b1 is None else b1
-        st = lib().sqo_step_range(self._dp, _ptr(pool), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g),
-                                  _ptr(o), _ptr(slots), b0, b1)
+        t0, t1 = (0, B * self.h_v) if tiles is None else tiles
+        args = (self._dp, _ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g), _ptr(o), _ptr(slots))
+        n = max(1, min(int(threads or 1), t1 - t0))
+        if n == 1:
+            return o, fn(*args, t0, t1)
+        cuts = [t0 + (t1 - t0) * i // n for i in range(n + 1)]
+        with ThreadPoolExecutor(n) as ex:  # ctypes releases the GIL during each call
+            sts = list(ex.map(lambda i: fn(*args, cuts[i], cuts[i + 1]), range(n)))
+        st = 0
+        for x in sts:
+            st |= x
         return o, st
 
-    def step_fp32(self, S, q, k, v, beta, g, slots=None, b0=0, b1=None, o=None):
+    def step(self, pool, q, k, v, beta, g, slots=None, o=None, threads=1, tiles=None):
+        """Quantized decode step in place on ``pool``; returns (o, status).
+        ``tiles`` = (t0, t1) restricts the step to tiles t0 .. t1-1
+        (tile = request * h_v + head); ``threads`` splits them over host threads."""
+        return self._run_tiles(lib().sqo_step_tiles, pool, q, k, v, beta, g, slots, o, threads, tiles)
+
+    def step_fp32(self, S, q, k, v, beta, g, slots=None, o=None, threads=1, tiles=None):
         """Unquantized step in place on the fp32 pool S [n_slots, h_v, d, d]."""
         assert S.dtype == np.float32 and S.flags.c_contiguous
-        q, k, v, beta, g = (_c(x, np.float32) for x in (q, k, v, beta, g))
-        slots = _c(slots, np.int32)
-        B = q.shape[0]
-        if o is None:
-            o = np.zeros((B, self.h_v, self.d), dtype=np.float32)
-        b1 = B if b1 is None else b1
-        st = lib().sqo_step_fp32_range(self._dp, _ptr(S), _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(g),
-                                       _ptr(o), _ptr(slots), b0, b1)
-        return o, st
+        return self._run_tiles(lib().sqo_step_fp32_tiles, S, q, k, v, beta, g, slots, o, threads, tiles)
 
     # ------------------------------------------------ record inspection
     def record(self, pool, slot, h):

@@ -348,29 +348,29 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
 
 /* ------------------------------------------------------ public entry */
 
-/* One decode step for batch rows [b0, b1) of a quantized pool. Inputs:
+/* One decode step for the tiles t in [t0, t1) (tile t = request t / h_v,
+ * value head t % h_v) of a batch of B requests in a quantized pool. Inputs:
  * q, k [B, h_k, d]; v [B, h_v, d]; beta [B, h_v]; g [B, h_v] (GDN) or
  * [B, h_v, d] (KDA); o [B, h_v, d]; slots [B] or NULL (identity). Returns
  * the status bits. Tiles of a skipped slot write o = 0. */
-uint32_t sqo_step_range(const sqo_desc *D, uint8_t *pool, const float *q, const float *k,
+uint32_t sqo_step_tiles(const sqo_desc *D, uint8_t *pool, const float *q, const float *k,
                         const float *v, const float *beta, const float *g, float *o,
-                        const int32_t *slots, int b0, int b1) {
+                        const int32_t *slots, int t0, int t1) {
   int d = D->d;
   float *T = malloc(sizeof(float) * d * d);
   float *gbuf = malloc(sizeof(float) * d);
   float *w = malloc(sizeof(float) * d);
   uint32_t st = 0;
   size_t slot_bytes = sqo_slot_bytes(D);
-  for (int b = b0; b < b1; b++) {
+  for (int t = t0; t < t1; t++) {
+    int b = t / D->h_v, h = t % D->h_v;
     int s = slot_of(D, slots, b, &st);
-    for (int h = 0; h < D->h_v; h++) {
-      if (s < 0) {
-        memset(o + ((size_t)b * D->h_v + h) * d, 0, sizeof(float) * d);
-        continue;
-      }
-      uint8_t *rec = pool + (size_t)s * slot_bytes + sqo_head_offset(D, h);
-      st |= step_tile(D, rec, b, h, q, k, v, beta, g, o, T, gbuf, w);
+    if (s < 0) {
+      memset(o + ((size_t)b * D->h_v + h) * d, 0, sizeof(float) * d);
+      continue;
     }
+    uint8_t *rec = pool + (size_t)s * slot_bytes + sqo_head_offset(D, h);
+    st |= step_tile(D, rec, b, h, q, k, v, beta, g, o, T, gbuf, w);
   }
   free(T); free(gbuf); free(w);
   return st;
@@ -379,7 +379,7 @@ uint32_t sqo_step_range(const sqo_desc *D, uint8_t *pool, const float *q, const 
 uint32_t sqo_step(const sqo_desc *D, uint8_t *pool, const float *q, const float *k,
                   const float *v, const float *beta, const float *g, float *o,
                   const int32_t *slots, int B) {
-  return sqo_step_range(D, pool, q, k, v, beta, g, o, slots, 0, B);
+  return sqo_step_tiles(D, pool, q, k, v, beta, g, o, slots, 0, B * D->h_v);
 }
 
 /* Quantize fp32 states S [B, h_v, d, d] (S-space) into the pool slots:
@@ -429,44 +429,44 @@ uint32_t sqo_dequantize(const sqo_desc *D, const uint8_t *pool, float *S, const 
   return st;
 }
 
-/* Unquantized FP32 state step (S-space), S pool [n_slots, h_v, d, d]:
+/* Unquantized FP32 state step (S-space) for tiles [t0, t1), S pool
+ * [n_slots, h_v, d, d]:
  *   G = g_i S_ij ; P_j = sum_i G_ij k_i ; u_j = beta (v_j - P_j) ;
  *   S'_ij = fmaf(k_i, u_j, G_ij) ; o_j = sum_i S'_ij q_i. */
-uint32_t sqo_step_fp32_range(const sqo_desc *D, float *Spool, const float *q_all, const float *k_all,
+uint32_t sqo_step_fp32_tiles(const sqo_desc *D, float *Spool, const float *q_all, const float *k_all,
                              const float *v_all, const float *beta_all, const float *g_all, float *o_all,
-                             const int32_t *slots, int b0, int b1) {
+                             const int32_t *slots, int t0, int t1) {
   int d = D->d;
   float *gbuf = malloc(sizeof(float) * d);
   float *u = malloc(sizeof(float) * d);
   uint32_t st = 0;
-  for (int b = b0; b < b1; b++) {
+  for (int t = t0; t < t1; t++) {
+    int b = t / D->h_v, h = t % D->h_v;
     int s = slot_of(D, slots, b, &st);
-    for (int h = 0; h < D->h_v; h++) {
-      float *o = o_all + ((size_t)b * D->h_v + h) * d;
-      if (s < 0) { memset(o, 0, sizeof(float) * d); continue; }
-      int hk = h / (D->h_v / D->h_k);
-      const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
-      const float *k = k_all + ((size_t)b * D->h_k + hk) * d;
-      const float *v = v_all + ((size_t)b * D->h_v + h) * d;
-      float beta = beta_all[(size_t)b * D->h_v + h];
-      const float *gate = gate_vector(D, g_all, b, h, gbuf);
-      float *S = Spool + ((size_t)s * D->h_v + h) * d * d;
-      for (int i = 0; i < d; i++)
-        for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
-      for (int j = 0; j < d; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)k[i];
-        float P = (float)acc;
-        u[j] = beta * (v[j] - P);
-      }
-      for (int i = 0; i < d; i++)
-        for (int j = 0; j < d; j++) S[i * d + j] = fmaf(k[i], u[j], S[i * d + j]);
-      for (int j = 0; j < d; j++) {
-        double acc = 0.0;
-        for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)q[i];
-        o[j] = (float)acc;
-        if (isnan(o[j])) st |= ST_NAN;
-      }
+    float *o = o_all + ((size_t)b * D->h_v + h) * d;
+    if (s < 0) { memset(o, 0, sizeof(float) * d); continue; }
+    int hk = h / (D->h_v / D->h_k);
+    const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
+    const float *k = k_all + ((size_t)b * D->h_k + hk) * d;
+    const float *v = v_all + ((size_t)b * D->h_v + h) * d;
+    float beta = beta_all[(size_t)b * D->h_v + h];
+    const float *gate = gate_vector(D, g_all, b, h, gbuf);
+    float *S = Spool + ((size_t)s * D->h_v + h) * d * d;
+    for (int i = 0; i < d; i++)
+      for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
+    for (int j = 0; j < d; j++) {
+      double acc = 0.0;
+      for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)k[i];
+      float P = (float)acc;
+      u[j] = beta * (v[j] - P);
+    }
+    for (int i = 0; i < d; i++)
+      for (int j = 0; j < d; j++) S[i * d + j] = fmaf(k[i], u[j], S[i * d + j]);
+    for (int j = 0; j < d; j++) {
+      double acc = 0.0;
+      for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)q[i];
+      o[j] = (float)acc;
+      if (isnan(o[j])) st |= ST_NAN;
     }
   }
   free(gbuf); free(u);
@@ -475,5 +475,5 @@ uint32_t sqo_step_fp32_range(const sqo_desc *D, float *Spool, const float *q_all
 
 uint32_t sqo_step_fp32(const sqo_desc *D, float *Spool, const float *q, const float *k, const float *v,
                        const float *beta, const float *g, float *o, const int32_t *slots, int B) {
-  return sqo_step_fp32_range(D, Spool, q, k, v, beta, g, o, slots, 0, B);
+  return sqo_step_fp32_tiles(D, Spool, q, k, v, beta, g, o, slots, 0, B * D->h_v);
 }

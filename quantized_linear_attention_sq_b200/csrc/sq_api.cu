@@ -1,0 +1,463 @@
+// sq_api.cu -- host side of the C ABI declared in include/sq.h: argument
+// validation, record layout, device tables and kernel launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "sq.h"
+#include "sq_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sq_status fail(sq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+sq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+uint64_t round_up(uint64_t x, uint64_t m) { return (x + m - 1) / m * m; }
+
+}  // namespace
+
+struct sq_handle {
+  sq_state_desc desc{};
+  int d = 0;
+  int device = 0;
+  int num_sms = 0;
+  // host copies of the layout
+  std::vector<uint32_t> rec_off, rec_bytes;
+  std::vector<uint16_t> row_off;
+  std::vector<uint8_t> row_code;
+  uint64_t slot_bytes = 0, pool_bytes = 0, max_rec = 0;
+  // device tables (one allocation)
+  void* dev_block = nullptr;
+  sqk::Tables tables{};
+  // launch configuration of the step kernel
+  int step_grid = 0;
+  int nstage = 0;
+  uint32_t rec_cap = 0, stage_bytes = 0;
+  size_t step_smem = 0;
+  uint64_t launches = 0;
+};
+
+namespace {
+
+template <int D>
+constexpr int threads_for() { return sqk::Geo<D>::NT; }
+
+int threads_of(int d) {
+  switch (d) {
+    case 128: return threads_for<128>();
+    case 64: return threads_for<64>();
+    default: return threads_for<32>();
+  }
+}
+
+// Every kernel that takes dynamic shared memory is allowed the device
+// maximum once; occupancy then depends only on what a launch asks for, so
+// handles with different record sizes never undo each other's setting.
+template <typename K>
+cudaError_t allow_max_smem(K kernel, int max_smem) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+}
+
+template <int D>
+cudaError_t allow_all(int max_smem) {
+  cudaError_t e = allow_max_smem(sqk::k_decode_step<D, true>, max_smem);
+  if (e == cudaSuccess) e = allow_max_smem(sqk::k_decode_step<D, false>, max_smem);
+  if (e == cudaSuccess) e = allow_max_smem(sqk::k_quantize<D>, max_smem);
+  if (e == cudaSuccess) e = allow_max_smem(sqk::k_dequantize<D>, max_smem);
+  return e;
+}
+
+template <int D, bool PACKED>
+cudaError_t occupancy(int* blocks, size_t smem) {
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, sqk::k_decode_step<D, PACKED>, sqk::Geo<D>::NT,
+                                                       smem);
+}
+
+// Choose stages and grid for the persistent step kernel.
+sq_status plan_step(sq_handle* h) {
+  const int d = h->d;
+  const bool packed = h->desc.fmt == SQ_FMT_PACKED;
+  const uint32_t rec = packed ? (uint32_t)h->max_rec : (uint32_t)(4u * d * d);
+  h->rec_cap = (uint32_t)round_up(rec, 128);
+  h->stage_bytes = (uint32_t)round_up(h->rec_cap + 31u * d, 128);
+  const int NG = d == 128 ? 32 : 32;  // row groups: 32 for every supported d
+  const size_t red = (size_t)NG * d * 4;
+  int dev_max_smem = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&dev_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  int sm_smem = 0;
+  e = cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, h->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  // target: 2 CTAs per SM for the packed kernel, 1 for fp32; 2..4 stages
+  const int want_ctas = packed ? 2 : 1;
+  const size_t static_smem = 2048;  // barriers, w vector, flags (upper bound)
+  const size_t budget = (size_t)sm_smem / want_ctas - static_smem - 1024 /* per-CTA reserve */;
+  int ns = (int)((budget - red) / h->stage_bytes);
+  if (ns > 4) ns = 4;
+  if (ns < 1) ns = 1;
+  size_t smem = (size_t)ns * h->stage_bytes + red;
+  while (smem > (size_t)dev_max_smem && ns > 1) {
+    --ns;
+    smem = (size_t)ns * h->stage_bytes + red;
+  }
+  if (smem > (size_t)dev_max_smem) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
+  h->nstage = ns;
+  h->step_smem = smem;
+  int blocks = 0;
+  if (d == 128) e = allow_all<128>(dev_max_smem);
+  else if (d == 64) e = allow_all<64>(dev_max_smem);
+  else e = allow_all<32>(dev_max_smem);
+  if (e != cudaSuccess) return cuda_fail(e, "kernel attributes");
+  if (d == 128) e = packed ? occupancy<128, true>(&blocks, smem) : occupancy<128, false>(&blocks, smem);
+  else if (d == 64) e = packed ? occupancy<64, true>(&blocks, smem) : occupancy<64, false>(&blocks, smem);
+  else e = packed ? occupancy<32, true>(&blocks, smem) : occupancy<32, false>(&blocks, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+  if (blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+  h->step_grid = blocks * h->num_sms;
+  return SQ_OK;
+}
+
+sq_status validate_desc(const sq_state_desc* d) {
+  if (!d) return fail(SQ_ERR_INVALID_ARG, "desc is NULL");
+  if (d->n_slots < 1) return fail(SQ_ERR_INVALID_ARG, "n_slots must be >= 1 (got %d)", d->n_slots);
+  if (d->h_v < 1 || d->h_k < 1) return fail(SQ_ERR_INVALID_ARG, "h_v and h_k must be >= 1");
+  if (d->h_v % d->h_k != 0) return fail(SQ_ERR_INVALID_ARG, "h_v (%d) must be a multiple of h_k (%d)", d->h_v, d->h_k);
+  if (d->d_k != d->d_v) return fail(SQ_ERR_UNSUPPORTED, "d_k != d_v is not supported");
+  if (d->d_k != 32 && d->d_k != 64 && d->d_k != 128)
+    return fail(SQ_ERR_UNSUPPORTED, "d must be 32, 64 or 128 (got %d)", d->d_k);
+  if (d->fmt != SQ_FMT_FP32 && d->fmt != SQ_FMT_PACKED) return fail(SQ_ERR_INVALID_ARG, "bad fmt %d", d->fmt);
+  if (d->gate != SQ_GATE_HEAD && d->gate != SQ_GATE_KEY_CHANNEL) return fail(SQ_ERR_INVALID_ARG, "bad gate %d", d->gate);
+  return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sq_last_error(void) { return g_last_error.c_str(); }
+
+const char* sq_version(void) { return "sq-b200 0.1 (sm_100a)"; }
+
+sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void* stream, sq_handle** out,
+                         size_t* pool_bytes) {
+  g_last_error.clear();
+  if (!out) return fail(SQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  sq_status s = validate_desc(desc);
+  if (s != SQ_OK) return s;
+  const int d = desc->d_k;
+  const int hv = desc->h_v;
+  const bool packed = desc->fmt == SQ_FMT_PACKED;
+  const bool per_row = desc->gate == SQ_GATE_KEY_CHANNEL;
+  const size_t n_units = per_row ? (size_t)hv * d : (size_t)hv;
+  if (packed) {
+    if (!calib || !calib->unit_bits || !calib->pivot_mask || !calib->col_scale || !calib->row_impact)
+      return fail(SQ_ERR_INVALID_ARG, "packed format needs all four calibration arrays");
+    for (size_t u = 0; u < n_units; ++u) {
+      const int b = calib->unit_bits[u];
+      if (!calib->pivot_mask[u] && b != 2 && b != 4 && b != 6 && b != 8)
+        return fail(SQ_ERR_INVALID_ARG, "unit %zu: bit width %d not in {2,4,6,8}", u, b);
+    }
+    for (size_t x = 0; x < (size_t)hv * d; ++x) {
+      const float c = calib->col_scale[x], p = calib->row_impact[x];
+      if (!std::isfinite(c) || !(c > 0.0f)) return fail(SQ_ERR_INVALID_ARG, "col_scale[%zu] = %g is not finite > 0", x, c);
+      if (!std::isfinite(p) || !(p > 0.0f)) return fail(SQ_ERR_INVALID_ARG, "row_impact[%zu] = %g is not finite > 0", x, p);
+      if (!std::isfinite(1.0f / c)) return fail(SQ_ERR_INVALID_ARG, "col_scale[%zu] = %g has no finite inverse", x, c);
+    }
+  }
+  sq_handle* h = new sq_handle();
+  h->desc = *desc;
+  h->d = d;
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e, "no usable CUDA device");
+  }
+  // ---- layout
+  h->rec_off.resize(hv);
+  h->rec_bytes.resize(hv);
+  h->row_off.assign((size_t)hv * d, 0);
+  h->row_code.assign((size_t)hv * d, 0);
+  uint64_t off = 0;
+  for (int hh = 0; hh < hv; ++hh) {
+    uint64_t n = 2ull * d;
+    for (int i = 0; i < d; ++i) {
+      const size_t u = per_row ? (size_t)hh * d + i : (size_t)hh;
+      uint8_t code;
+      uint64_t rb;
+      if (!packed) {
+        code = sqk::ROW_PIVOT;
+        rb = 0;
+      } else if (calib->pivot_mask[u]) {
+        code = sqk::ROW_PIVOT;
+        rb = 2ull * d;
+      } else {
+        code = (uint8_t)calib->unit_bits[u];
+        rb = (uint64_t)d * code / 8;
+      }
+      h->row_off[(size_t)hh * d + i] = (uint16_t)n;
+      h->row_code[(size_t)hh * d + i] = code;
+      n += rb;
+    }
+    n = round_up(n, 16);
+    if (!packed) n = 4ull * d * d;
+    h->rec_off[hh] = (uint32_t)off;
+    h->rec_bytes[hh] = (uint32_t)n;
+    if (n > h->max_rec) h->max_rec = n;
+    off += n;
+  }
+  h->slot_bytes = off;
+  h->pool_bytes = off * (uint64_t)desc->n_slots;
+  // ---- device tables: rec_off, rec_bytes [hv] u32; col, icol, phi [hv*d] f32;
+  //      row_off [hv*d] u16; row_code [hv*d] u8; status u32
+  const size_t nhd = (size_t)hv * d;
+  size_t o_rec_off = 0;
+  size_t o_rec_bytes = round_up(o_rec_off + 4 * hv, 16);
+  size_t o_col = round_up(o_rec_bytes + 4 * hv, 16);
+  size_t o_icol = round_up(o_col + 4 * nhd, 16);
+  size_t o_phi = round_up(o_icol + 4 * nhd, 16);
+  size_t o_row_off = round_up(o_phi + 4 * nhd, 16);
+  size_t o_row_code = round_up(o_row_off + 2 * nhd, 16);
+  size_t o_status = round_up(o_row_code + nhd, 16);
+  size_t total = round_up(o_status + 16, 256);
+  std::vector<uint8_t> host(total, 0);
+  memcpy(host.data() + o_rec_off, h->rec_off.data(), 4 * hv);
+  memcpy(host.data() + o_rec_bytes, h->rec_bytes.data(), 4 * hv);
+  float* col = reinterpret_cast<float*>(host.data() + o_col);
+  float* icol = reinterpret_cast<float*>(host.data() + o_icol);
+  float* phi = reinterpret_cast<float*>(host.data() + o_phi);
+  for (size_t x = 0; x < nhd; ++x) {
+    col[x] = packed ? calib->col_scale[x] : 1.0f;
+    volatile float c = col[x];
+    icol[x] = 1.0f / c;  // IEEE single-precision division
+    phi[x] = packed ? calib->row_impact[x] : 1.0f;
+  }
+  memcpy(host.data() + o_row_off, h->row_off.data(), 2 * nhd);
+  memcpy(host.data() + o_row_code, h->row_code.data(), nhd);
+  e = cudaMalloc(&h->dev_block, total);
+  if (e != cudaSuccess) {
+    delete h;
+    return fail(SQ_ERR_OOM, "cudaMalloc of %zu table bytes failed: %s", total, cudaGetErrorString(e));
+  }
+  e = cudaMemcpyAsync(h->dev_block, host.data(), total, cudaMemcpyHostToDevice, as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) {
+    cudaFree(h->dev_block);
+    delete h;
+    return cuda_fail(e, "uploading tables");
+  }
+  uint8_t* base = static_cast<uint8_t*>(h->dev_block);
+  h->tables.rec_off = reinterpret_cast<const uint32_t*>(base + o_rec_off);
+  h->tables.rec_bytes = reinterpret_cast<const uint32_t*>(base + o_rec_bytes);
+  h->tables.col = reinterpret_cast<const float*>(base + o_col);
+  h->tables.icol = reinterpret_cast<const float*>(base + o_icol);
+  h->tables.phi = reinterpret_cast<const float*>(base + o_phi);
+  h->tables.row_off = reinterpret_cast<const uint16_t*>(base + o_row_off);
+  h->tables.row_code = reinterpret_cast<const uint8_t*>(base + o_row_code);
+  h->tables.status = reinterpret_cast<uint32_t*>(base + o_status);
+  s = plan_step(h);
+  if (s != SQ_OK) {
+    cudaFree(h->dev_block);
+    delete h;
+    return s;
+  }
+  *out = h;
+  if (pool_bytes) *pool_bytes = (size_t)h->pool_bytes;
+  return SQ_OK;
+}
+
+sq_status sq_state_free(sq_handle* h) {
+  g_last_error.clear();
+  if (!h) return SQ_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaError_t e2 = cudaFree(h->dev_block);
+  delete h;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  if (e2 != cudaSuccess) return cuda_fail(e2, "cudaFree");
+  return SQ_OK;
+}
+
+sq_status sq_state_bytes(const sq_handle* h, sq_bytes_report* out) {
+  if (!h || !out) return fail(SQ_ERR_INVALID_ARG, "NULL argument");
+  const sq_state_desc& d = h->desc;
+  out->pool_bytes = h->pool_bytes;
+  out->slot_bytes = h->slot_bytes;
+  out->state_bytes_per_step = 2 * h->slot_bytes;
+  const uint64_t dd = (uint64_t)h->d;
+  const uint64_t g = d.gate == SQ_GATE_HEAD ? 1 : dd;
+  out->act_bytes_per_step = 4 * (2 * (uint64_t)d.h_k * dd + (uint64_t)d.h_v * dd + (uint64_t)d.h_v +
+                                 (uint64_t)d.h_v * g + (uint64_t)d.h_v * dd);
+  out->bits_per_value = 8.0 * (double)h->slot_bytes / ((double)d.h_v * dd * dd);
+  out->max_record_bytes = h->max_rec;
+  return SQ_OK;
+}
+
+sq_status sq_head_layout(const sq_handle* h, int32_t head, uint64_t* offset, uint64_t* record_bytes) {
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (head < 0 || head >= h->desc.h_v) return fail(SQ_ERR_INVALID_ARG, "head %d out of range", head);
+  if (offset) *offset = h->rec_off[head];
+  if (record_bytes) *record_bytes = h->rec_bytes[head];
+  return SQ_OK;
+}
+
+uint64_t sq_launch_count(const sq_handle* h) { return h ? h->launches : 0; }
+
+sq_status sq_get_status(sq_handle* h, void* stream, uint32_t* bits, int32_t clear) {
+  g_last_error.clear();
+  if (!h || !bits) return fail(SQ_ERR_INVALID_ARG, "NULL argument");
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, h->tables.status, 4, cudaMemcpyDeviceToHost, as_stream(stream));
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(h->tables.status, 0, 4, as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  *bits = v;
+  return SQ_OK;
+}
+
+#define SQ_CHECK_PTR(p, name)                                                               \
+  do {                                                                                      \
+    if (!(p)) return fail(SQ_ERR_INVALID_ARG, "%s is NULL", name);                         \
+    if (!aligned16(p)) return fail(SQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* k, const float* v, const float* beta,
+                         const float* g, float* o, const int32_t* slot_ids, int32_t B, void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (B == 0) return SQ_OK;
+  if ((int64_t)B * h->desc.h_v > (int64_t)INT32_MAX / 2) return fail(SQ_ERR_INVALID_ARG, "B too large");
+  SQ_CHECK_PTR(pool, "pool");
+  SQ_CHECK_PTR(q, "q");
+  SQ_CHECK_PTR(k, "k");
+  SQ_CHECK_PTR(v, "v");
+  SQ_CHECK_PTR(o, "o");
+  if (!beta) return fail(SQ_ERR_INVALID_ARG, "beta is NULL");
+  if (!g) return fail(SQ_ERR_INVALID_ARG, "g is NULL");
+  if (h->desc.gate == SQ_GATE_KEY_CHANNEL && !aligned16(g)) return fail(SQ_ERR_INVALID_ARG, "g is not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(SQ_ERR_INVALID_ARG, "beta/g not 4-byte aligned");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  sqk::StepArgs a{};
+  a.pool = static_cast<uint8_t*>(pool);
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
+  a.slots = slot_ids;
+  a.B = B; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots; a.gate_kind = h->desc.gate;
+  a.nstage = h->nstage; a.rec_cap = h->rec_cap; a.stage_bytes = h->stage_bytes;
+  a.slot_bytes = h->slot_bytes;
+  a.t = h->tables;
+  const int n_tiles = B * h->desc.h_v;
+  const int grid = n_tiles < h->step_grid ? n_tiles : h->step_grid;
+  const int nt = threads_of(h->d);
+  cudaStream_t st = as_stream(stream);
+  const bool packed = h->desc.fmt == SQ_FMT_PACKED;
+  if (packed) {
+    if (h->d == 128) sqk::k_decode_step<128, true><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step<64, true><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step<32, true><<<grid, nt, h->step_smem, st>>>(a);
+  } else {
+    if (h->d == 128) sqk::k_decode_step<128, false><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step<64, false><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step<32, false><<<grid, nt, h->step_smem, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching the decode step");
+  h->launches++;
+  return SQ_OK;
+}
+
+sq_status sq_quantize_state(sq_handle* h, void* pool, const float* S, const int32_t* slot_ids, int32_t B,
+                            void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (B == 0) return SQ_OK;
+  SQ_CHECK_PTR(pool, "pool");
+  SQ_CHECK_PTR(S, "S");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  cudaStream_t st = as_stream(stream);
+  const int n_tiles = B * h->desc.h_v;
+  const int nt = threads_of(h->d);
+  if (h->desc.fmt == SQ_FMT_FP32) {
+    if (h->d == 128) sqk::k_copy_fp32<128><<<n_tiles, 256, 0, st>>>(static_cast<float*>(pool), S, nullptr, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+    else if (h->d == 64) sqk::k_copy_fp32<64><<<n_tiles, 256, 0, st>>>(static_cast<float*>(pool), S, nullptr, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+    else sqk::k_copy_fp32<32><<<n_tiles, 256, 0, st>>>(static_cast<float*>(pool), S, nullptr, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+  } else {
+    sqk::QuantArgs a{};
+    a.pool = static_cast<uint8_t*>(pool);
+    a.S = S;
+    a.slots = slot_ids;
+    a.B = B; a.h_v = h->desc.h_v; a.n_slots = h->desc.n_slots;
+    a.slot_bytes = h->slot_bytes;
+    a.t = h->tables;
+    const size_t smem = round_up(h->max_rec, 16) + 7 * (size_t)h->d;
+    if (h->d == 128) sqk::k_quantize<128><<<n_tiles, nt, smem, st>>>(a);
+    else if (h->d == 64) sqk::k_quantize<64><<<n_tiles, nt, smem, st>>>(a);
+    else sqk::k_quantize<32><<<n_tiles, nt, smem, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching quantize");
+  h->launches++;
+  return SQ_OK;
+}
+
+sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, const int32_t* slot_ids, int32_t B,
+                              void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (B == 0) return SQ_OK;
+  SQ_CHECK_PTR(pool, "pool");
+  SQ_CHECK_PTR(S_out, "S_out");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  cudaStream_t st = as_stream(stream);
+  const int n_tiles = B * h->desc.h_v;
+  const int nt = threads_of(h->d);
+  if (h->desc.fmt == SQ_FMT_FP32) {
+    float* P = const_cast<float*>(static_cast<const float*>(pool));
+    if (h->d == 128) sqk::k_copy_fp32<128><<<n_tiles, 256, 0, st>>>(P, nullptr, S_out, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+    else if (h->d == 64) sqk::k_copy_fp32<64><<<n_tiles, 256, 0, st>>>(P, nullptr, S_out, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+    else sqk::k_copy_fp32<32><<<n_tiles, 256, 0, st>>>(P, nullptr, S_out, slot_ids, h->desc.h_v, h->desc.n_slots, h->tables.status);
+  } else {
+    sqk::QuantArgs a{};
+    a.pool = static_cast<uint8_t*>(const_cast<void*>(pool));
+    a.S_out = S_out;
+    a.slots = slot_ids;
+    a.B = B; a.h_v = h->desc.h_v; a.n_slots = h->desc.n_slots;
+    a.slot_bytes = h->slot_bytes;
+    a.t = h->tables;
+    const size_t smem = round_up(h->max_rec, 16);
+    if (h->d == 128) sqk::k_dequantize<128><<<n_tiles, nt, smem, st>>>(a);
+    else if (h->d == 64) sqk::k_dequantize<64><<<n_tiles, nt, smem, st>>>(a);
+    else sqk::k_dequantize<32><<<n_tiles, nt, smem, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching dequantize");
+  h->launches++;
+  return SQ_OK;
+}
+
+}  // extern "C"
