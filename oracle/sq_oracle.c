@@ -30,27 +30,30 @@
  *
  * The pages fix the method but not its arithmetic; the canonical
  * elementwise arithmetic below is this project's reading, chosen so that
- * two implementations agree bit for bit on the integer codes. Reductions
- * (the two dot products per column) are the only order-free steps: here
- * they are accumulated in fp64 from exact fp32 products and rounded once.
+ * two implementations agree bit for bit on the integer codes. The only sums
+ * are the two column dot products; each is taken from exact products and
+ * rounded once to fp32 (here: exact products and an extended-precision
+ * accumulator). S^T k is the one sum that feeds back into the state, so it
+ * is the one whose rounding decides reproducibility over a long rollout.
  *
  * Column-normalised form. With S = T diag(c), the whole step is carried out
  * on T (the row-scale x code part), and c enters only where S^T k and S^T q
- * are formed and where u is mapped back to T units:
- *   1. a_i   = fp32(r_i * g_i)                          (quantized rows)
- *   2. T_ij  = fp32(q_ij * a_i)        quantized rows
- *      T_ij  = fp32(h_ij * g_i)        pivot rows (h = stored fp16 of T)
- *   3. P_j   = sum_i T_ij k_i          (fp64 sum, rounded once to fp32)
- *   4. p_j = fp32(c_j P_j); u_j = fp32(beta fp32(v_j - p_j));
+ * are formed and where u is mapped back to T units. A row is stored as
+ * values V_ij with a per-row multiplier M_i, the gated T being V_ij M_i:
+ *   1. quantized rows: V = integer code q_ij, M_i = a_i = fp32(r_i * g_i)
+ *      pivot rows:     V = stored fp16 value h_ij of T, M_i = g_i
+ *   2. P_j   = sum_i V_ij M_i k_i  (the exact value, rounded once to fp32)
+ *   3. p_j = fp32(c_j P_j); u_j = fp32(beta fp32(v_j - p_j));
  *      w_j = fp32(u_j * ic_j) with ic_j = fp32(1 / c_j)
- *   5. T'_ij = fmaf(k_i, w_j, T_ij)
- *   6. O_j   = sum_i T'_ij q_i (fp64, rounded once); o_j = fp32(c_j O_j)
- *   7. m_i   = max_j |T'_ij| (a NaN makes m_i NaN)
- *   8. s_i   = fp32(fp32(phi_i m_i) / qmax_i); r'_i = fp16 of s_i rounded
+ *   4. T'_ij = fmaf(V_ij, M_i, fp32(k_i * w_j))   (gate, decay and update,
+ *      one rounding of the exact gated value plus the rounded update)
+ *   5. O_j   = sum_i T'_ij q_i (exact, rounded once); o_j = fp32(c_j O_j)
+ *   6. m_i   = max_j |T'_ij| (a NaN makes m_i NaN)
+ *   7. s_i   = fp32(fp32(phi_i m_i) / qmax_i); r'_i = fp16 of s_i rounded
  *      toward +inf (saturating at 65504); ir_i = 0 if r'_i == 0 else
  *      fp32(1 / r'_i)
- *   9. q'_ij = RNE(min(max(fp32(T'_ij * ir_i), -qmax), qmax))
- *  10. pivot rows: h'_ij = fp16 round-to-nearest-even of T'_ij, saturating
+ *   8. q'_ij = RNE(min(max(fp32(T'_ij * ir_i), -qmax), qmax))
+ *   9. pivot rows: h'_ij = fp16 round-to-nearest-even of T'_ij, saturating
  *      at +-65504; a NaN stores 0.
  *  A row whose m_i is NaN stores r' = 0 and all codes 0 (status bit 0).
  *
@@ -215,29 +218,28 @@ static int qmax_of(int b) { return (1 << (b - 1)) - 1; }
 
 /* ------------------------------------------------ per-tile primitives */
 
-/* Read a head record into column-normalised T (d x d), applying the
- * per-row multiplier: a_i = r_i * g_i for quantized rows, g_i for pivots.
- * With gate == NULL the multiplier is r_i (quantized) and 1 (pivots), and no
- * rounding beyond the exact q * r product happens. */
-static void load_T(const sqo_desc *D, int h, const uint8_t *rec, const float *gate, float *T) {
+/* Read a head record as stored values V (d x d) and a per-row multiplier M,
+ * so that the gated, column-normalised state is exactly V_ij * M_i:
+ * quantized rows V = integer code, M = a_i = fp32(r_i * g_i); pivot rows
+ * V = the fp16 value, M = g_i. With gate == NULL the multiplier is r_i
+ * (quantized) and 1 (pivots). Nothing is rounded here. */
+static void load_VM(const sqo_desc *D, int h, const uint8_t *rec, const float *gate, float *V, float *M) {
   int d = D->d;
   for (int i = 0; i < d; i++) {
     const uint8_t *row = rec + row_offset(D, h, i);
     if (row_is_pivot(D, h, i)) {
-      for (int j = 0; j < d; j++) {
-        float hv = sqo_f16_to_f32(rd16(row + 2 * j));
-        T[i * d + j] = gate ? hv * gate[i] : hv;
-      }
+      M[i] = gate ? gate[i] : 1.0f;
+      for (int j = 0; j < d; j++) V[i * d + j] = sqo_f16_to_f32(rd16(row + 2 * j));
     } else {
       int b = row_width(D, h, i);
       float r = sqo_f16_to_f32(rd16(rec + 2 * i));
-      float a = gate ? r * gate[i] : r;
-      for (int j = 0; j < d; j++) T[i * d + j] = (float)sqo_get_code(row, b, j) * a;
+      M[i] = gate ? r * gate[i] : r;
+      for (int j = 0; j < d; j++) V[i * d + j] = (float)sqo_get_code(row, b, j);
     }
   }
 }
 
-/* Steps 7-10: requantize column-normalised T' into the record. */
+/* Steps 6-9: requantize column-normalised T' into the record. */
 static uint32_t store_T(const sqo_desc *D, int h, uint8_t *rec, const float *T) {
   int d = D->d;
   uint32_t st = 0;
@@ -311,7 +313,7 @@ static int slot_of(const sqo_desc *D, const int32_t *slots, int b, uint32_t *st)
 static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
                           const float *q_all, const float *k_all, const float *v_all,
                           const float *beta_all, const float *g_all, float *o_all,
-                          float *T, float *gbuf, float *w) {
+                          float *T, float *M, float *gbuf, float *w) {
   int d = D->d;
   int hk = h / (D->h_v / D->h_k);
   const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
@@ -323,26 +325,30 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
   const float *gate = gate_vector(D, g_all, b, h, gbuf);
   uint32_t st = 0;
 
-  load_T(D, h, rec, gate, T);                          /* steps 1-2 */
-  for (int j = 0; j < d; j++) {                        /* steps 3-4 */
-    double acc = 0.0;
-    for (int i = 0; i < d; i++) acc += (double)T[i * d + j] * (double)k[i];
+  load_VM(D, h, rec, gate, T, M);                      /* step 1 */
+  for (int j = 0; j < d; j++) {                        /* steps 2-3 */
+    /* each product V * M * k is exact in long double (at most 59 bits) */
+    long double acc = 0.0L;
+    for (int i = 0; i < d; i++) acc += (long double)T[i * d + j] * (long double)M[i] * (long double)k[i];
     float P = (float)acc;
     float p = c[j] * P;
     float u = beta * (v[j] - p);
     float ic = 1.0f / c[j];
     w[j] = u * ic;
   }
-  for (int i = 0; i < d; i++)                          /* step 5 */
-    for (int j = 0; j < d; j++) T[i * d + j] = fmaf(k[i], w[j], T[i * d + j]);
-  for (int j = 0; j < d; j++) {                        /* step 6 */
-    double acc = 0.0;
-    for (int i = 0; i < d; i++) acc += (double)T[i * d + j] * (double)q[i];
+  for (int i = 0; i < d; i++)                          /* step 4 */
+    for (int j = 0; j < d; j++) {
+      float kw = k[i] * w[j];
+      T[i * d + j] = fmaf(T[i * d + j], M[i], kw);
+    }
+  for (int j = 0; j < d; j++) {                        /* step 5 */
+    long double acc = 0.0L;
+    for (int i = 0; i < d; i++) acc += (long double)T[i * d + j] * (long double)q[i];
     float O = (float)acc;
     o[j] = c[j] * O;
     if (isnan(o[j])) st |= ST_NAN;
   }
-  st |= store_T(D, h, rec, T);                         /* steps 7-10 */
+  st |= store_T(D, h, rec, T);                         /* steps 6-9 */
   return st;
 }
 
@@ -358,6 +364,7 @@ uint32_t sqo_step_tiles(const sqo_desc *D, uint8_t *pool, const float *q, const 
                         const int32_t *slots, int t0, int t1) {
   int d = D->d;
   float *T = malloc(sizeof(float) * d * d);
+  float *M = malloc(sizeof(float) * d);
   float *gbuf = malloc(sizeof(float) * d);
   float *w = malloc(sizeof(float) * d);
   uint32_t st = 0;
@@ -370,9 +377,9 @@ uint32_t sqo_step_tiles(const sqo_desc *D, uint8_t *pool, const float *q, const 
       continue;
     }
     uint8_t *rec = pool + (size_t)s * slot_bytes + sqo_head_offset(D, h);
-    st |= step_tile(D, rec, b, h, q, k, v, beta, g, o, T, gbuf, w);
+    st |= step_tile(D, rec, b, h, q, k, v, beta, g, o, T, M, gbuf, w);
   }
-  free(T); free(gbuf); free(w);
+  free(T); free(M); free(gbuf); free(w);
   return st;
 }
 
@@ -383,7 +390,7 @@ uint32_t sqo_step(const sqo_desc *D, uint8_t *pool, const float *q, const float 
 }
 
 /* Quantize fp32 states S [B, h_v, d, d] (S-space) into the pool slots:
- * T_ij = fp32(S_ij * ic_j), then steps 7-10. */
+ * T_ij = fp32(S_ij * ic_j), then steps 6-9. */
 uint32_t sqo_quantize(const sqo_desc *D, uint8_t *pool, const float *S, const int32_t *slots, int B) {
   int d = D->d;
   float *T = malloc(sizeof(float) * d * d);
@@ -411,7 +418,8 @@ uint32_t sqo_quantize(const sqo_desc *D, uint8_t *pool, const float *S, const in
  * for quantized rows and fp32(h c_j) for pivot rows. Skipped slots give 0. */
 uint32_t sqo_dequantize(const sqo_desc *D, const uint8_t *pool, float *S, const int32_t *slots, int B) {
   int d = D->d;
-  float *T = malloc(sizeof(float) * d * d);
+  float *V = malloc(sizeof(float) * d * d);
+  float *M = malloc(sizeof(float) * d);
   uint32_t st = 0;
   size_t slot_bytes = sqo_slot_bytes(D);
   for (int b = 0; b < B; b++) {
@@ -420,12 +428,15 @@ uint32_t sqo_dequantize(const sqo_desc *D, const uint8_t *pool, float *S, const 
       float *Sh = S + ((size_t)b * D->h_v + h) * d * d;
       if (s < 0) { memset(Sh, 0, sizeof(float) * d * d); continue; }
       const float *c = D->col_scale + (size_t)h * d;
-      load_T(D, h, pool + (size_t)s * slot_bytes + sqo_head_offset(D, h), NULL, T);
+      load_VM(D, h, pool + (size_t)s * slot_bytes + sqo_head_offset(D, h), NULL, V, M);
       for (int i = 0; i < d; i++)
-        for (int j = 0; j < d; j++) Sh[i * d + j] = T[i * d + j] * c[j];
+        for (int j = 0; j < d; j++) {
+          float t = V[i * d + j] * M[i]; /* exact: at most 19 significant bits */
+          Sh[i * d + j] = t * c[j];
+        }
     }
   }
-  free(T);
+  free(V); free(M);
   return st;
 }
 
@@ -455,8 +466,8 @@ uint32_t sqo_step_fp32_tiles(const sqo_desc *D, float *Spool, const float *q_all
     for (int i = 0; i < d; i++)
       for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
     for (int j = 0; j < d; j++) {
-      double acc = 0.0;
-      for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)k[i];
+      long double acc = 0.0L;
+      for (int i = 0; i < d; i++) acc += (long double)S[i * d + j] * (long double)k[i];
       float P = (float)acc;
       u[j] = beta * (v[j] - P);
     }

@@ -77,7 +77,11 @@ int threads_of(int d) {
 // handles with different record sizes never undo each other's setting.
 template <typename K>
 cudaError_t allow_max_smem(K kernel, int max_smem) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              max_smem - (int)fa.sharedSizeBytes);
 }
 
 template <int D>
@@ -118,11 +122,12 @@ sq_status plan_step(sq_handle* h) {
   if (ns > 4) ns = 4;
   if (ns < 1) ns = 1;
   size_t smem = (size_t)ns * h->stage_bytes + red;
-  while (smem > (size_t)dev_max_smem && ns > 1) {
+  const size_t dyn_max = (size_t)dev_max_smem - 1024;  // room for the static shared variables
+  while (smem > dyn_max && ns > 1) {
     --ns;
     smem = (size_t)ns * h->stage_bytes + red;
   }
-  if (smem > (size_t)dev_max_smem) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
+  if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
   h->nstage = ns;
   h->step_smem = smem;
   int blocks = 0;

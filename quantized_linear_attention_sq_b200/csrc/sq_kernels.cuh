@@ -517,7 +517,12 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
           const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
           mul = __fmul_rn(R, gr[r]);
         }
-        load_row(row, code, cc, mul, T[r]);
+        // unpack through a temporary: writing T[r] from inside the width
+        // switch would push the whole tile into local memory
+        float2 tmp[8];
+        load_row(row, code, cc, mul, tmp);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) T[r][p] = tmp[p];
       } else {
         const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
 #pragma unroll

@@ -104,8 +104,14 @@ def compare_slots(o_: oracle.Oracle, ref: np.ndarray, got: np.ndarray, st: Stats
             off, nb = o_.layout.head_offset[h], o_.layout.record_bytes[h]
             if np.array_equal(a[off:off + nb], b[off:off + nb]):
                 continue
-            ca, cb = o_.codes(a, s, h), o_.codes(b, s, h)
-            ra, rb = o_.row_scales(a, s, h), o_.row_scales(b, s, h)
+            ca, cb = o_.codes(a, 0, h), o_.codes(b, 0, h)
+            ra, rb = o_.row_scales(a, 0, h), o_.row_scales(b, 0, h)
+            if len(st.notes) < 12:
+                rows = [i for i in range(d) if ra[i] != rb[i] or np.any(ca[i] != cb[i])]
+                i0 = rows[0]
+                st.notes.append(f"slot {s} head {h} kind {o_.row_kind(h, i0)} rows {rows[:6]} "
+                                f"r {ra[i0]}/{rb[i0]} codes {ca[i0][:6]}/{cb[i0][:6]} "
+                                f"ndiff {int((ca != cb).sum())}")
             found = 0
             for i in range(d):
                 piv, _ = o_.row_kind(h, i)
