@@ -106,8 +106,8 @@ sq_status plan_step(sq_handle* h) {
   const uint32_t rec = packed ? (uint32_t)h->max_rec : (uint32_t)(4u * d * d);
   h->rec_cap = (uint32_t)round_up(rec, 128);
   h->stage_bytes = (uint32_t)round_up(h->rec_cap + 31u * d, 128);
-  const int NG = d == 128 ? 32 : 32;  // row groups: 32 for every supported d
-  const size_t red = (size_t)NG * d * 4;
+  const int NG = 32;  // row groups per CTA: 32 for every supported d
+  const size_t red = (size_t)NG * d * (packed ? 8 : 4);  // fp64 column partials when packed
   int dev_max_smem = 0;
   cudaError_t e = cudaDeviceGetAttribute(&dev_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");

@@ -190,6 +190,72 @@ __device__ __forceinline__ void unpack16(const uint32_t* w, float2 (&f)[8]) {
   }
 }
 
+// Field j of a 16-code chunk placed at bits [20-B, 20) of the word
+// 0x3FF00000. Read as the high word of a double (low word 0) this is
+// 1 + field * 2^-B exactly; read as a float it is 1.875 + field * 2^-(B+3).
+// One shift (or funnel shift) and one LOP3 per field give both.
+template <int B>
+__device__ __forceinline__ uint32_t field_hi(const uint32_t* w, int j) {
+  constexpr int POS = 20 - B;
+  constexpr uint32_t MASK = ((1u << B) - 1u) << POS;
+  const int bit = B * j;
+  const int wi = bit >> 5;
+  const int sh = bit & 31;
+  uint32_t x;
+  if (sh + B <= 32)
+    x = sh >= POS ? (w[wi] >> (sh - POS)) : (w[wi] << (POS - sh));
+  else
+    x = __funnelshift_r(w[wi], w[wi + 1], sh - POS);  // a straddling field always has sh > POS
+  return 0x3FF00000u | (x & MASK);
+}
+
+// Pass-A unpack of one quantized 16-code chunk: the codes q as floats (exact)
+// and the high words of the doubles 1 + field * 2^-B that feed the fp64
+// column sum (with the per-row factor 2^B a k, minus 1.5 2^B a k per row,
+// they give q a k exactly up to fp64 rounding).
+template <int B>
+__device__ __forceinline__ void unpack_q_hi(const uint8_t* row, int cc, float2 (&V)[8], uint32_t (&xh)[16]) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(row + 2 * B * cc);
+  uint32_t w[B / 2];
+#pragma unroll
+  for (int i = 0; i < B / 2; ++i) w[i] = src[i];
+  const float S = (float)(1 << (B + 3));
+  const float C = 1.875f * S + (float)(1 << (B - 1));
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t h0 = field_hi<B>(w, 2 * p), h1 = field_hi<B>(w, 2 * p + 1);
+    xh[2 * p] = h0;
+    xh[2 * p + 1] = h1;
+    V[p] = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)), make_float2(S, S),
+                      make_float2(-C, -C));
+  }
+}
+
+// Pass-A unpack of one fp16 pivot chunk: the values as floats and the high
+// words of the same values as doubles (an fp16 value has a zero low word).
+__device__ __forceinline__ void unpack_pivot_hi(const uint8_t* row, int cc, float2 (&V)[8], uint32_t (&xh)[16]) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(row + 32 * cc);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    __half2 h2 = *reinterpret_cast<const __half2*>(src + p);
+    float2 x = __half22float2(h2);
+    V[p] = x;
+    xh[2 * p] = (uint32_t)__double2hiint((double)x.x);
+    xh[2 * p + 1] = (uint32_t)__double2hiint((double)x.y);
+  }
+}
+
+__device__ __forceinline__ void unpack_hi(const uint8_t* row, uint8_t code, int cc, float2 (&V)[8],
+                                          uint32_t (&xh)[16]) {
+  switch (code) {
+    case 8: unpack_q_hi<8>(row, cc, V, xh); break;
+    case 6: unpack_q_hi<6>(row, cc, V, xh); break;
+    case 4: unpack_q_hi<4>(row, cc, V, xh); break;
+    case 2: unpack_q_hi<2>(row, cc, V, xh); break;
+    default: unpack_pivot_hi(row, cc, V, xh); break;
+  }
+}
+
 // Pack 16 magic-number floats (2^23 + field) into b/2 words.
 template <int B>
 __device__ __forceinline__ void pack16(const uint32_t (&fb)[16], uint32_t* w) {
@@ -383,6 +449,34 @@ __device__ __forceinline__ float column_sum(float* red, int rg, int cc, const fl
   return tot;
 }
 
+// fp64 column sums (same scheme as column_sum); returns the total rounded
+// once to fp32 for threads < D.
+template <int D>
+__device__ __forceinline__ float column_sum_f64(double* red, int rg, int cc, const double (&part)[16]) {
+  using G = Geo<D>;
+  double2* dst = reinterpret_cast<double2*>(red + rg * D + 16 * cc);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) dst[p] = make_double2(part[2 * p], part[2 * p + 1]);
+  __syncthreads();
+  float tot = 0.0f;
+  if (threadIdx.x < D) {
+    const int j = threadIdx.x;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    int g = 0;
+#pragma unroll
+    for (; g + 3 < G::NG; g += 4) {
+      a0 += red[(g + 0) * D + j];
+      a1 += red[(g + 1) * D + j];
+      a2 += red[(g + 2) * D + j];
+      a3 += red[(g + 3) * D + j];
+    }
+#pragma unroll
+    for (; g < G::NG; ++g) a0 += red[g * D + j];
+    tot = __double2float_rn((a0 + a1) + (a2 + a3));
+  }
+  return tot;
+}
+
 // ================================================================ step kernel
 template <int D>
 __device__ __forceinline__ int tile_slot(const StepArgs& a, int b) {
@@ -501,29 +595,52 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
       gr[r] = a.gate_kind == 0 ? gh : S.g()[i];
     }
 
-    // ---- pass A: dequantize + gate, partial S^T k
+    // ---- pass A: values, gate, column sum S^T k
+    // packed: T holds the stored values V (codes or fp16) and mr the per-row
+    // multiplier M (a_i = r_i g_i, or g_i for a pivot row); the column sum
+    // is accumulated in fp64 from the exact per-row factors (see unpack_hi).
+    // fp32: T holds the gated state g_i S_ij and the column sum is fp32.
     float2 T[G::RPT][8];
+    float mr[G::RPT];
     float2 part[8];
+    float P;
+    if (PACKED) {
+      double acc[16];
 #pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const int i = r * G::NG + rg;
-      if (PACKED) {
+      for (int j = 0; j < 16; ++j) acc[j] = 0.0;
+      double off = 0.0;
+#pragma unroll
+      for (int r = 0; r < G::RPT; ++r) {
+        const int i = r * G::NG + rg;
         const uint8_t code = S.row_code()[i];
         const uint8_t* row = S.rec() + S.row_off()[i];
-        float mul;
+        double kap;
         if (code == ROW_PIVOT) {
-          mul = gr[r];
+          mr[r] = gr[r];
+          kap = (double)gr[r] * (double)kr[r];
         } else {
           const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
-          mul = __fmul_rn(R, gr[r]);
+          mr[r] = __fmul_rn(R, gr[r]);
+          kap = (double)mr[r] * (double)kr[r] * (double)(1 << code);
+          off = off + 1.5 * kap;
         }
-        // unpack through a temporary: writing T[r] from inside the width
+        // unpack through temporaries: writing T[r] from inside the width
         // switch would push the whole tile into local memory
-        float2 tmp[8];
-        load_row(row, code, cc, mul, tmp);
+        float2 vt[8];
+        uint32_t xh[16];
+        unpack_hi(row, code, cc, vt, xh);
 #pragma unroll
-        for (int p = 0; p < 8; ++p) T[r][p] = tmp[p];
-      } else {
+        for (int p = 0; p < 8; ++p) T[r][p] = vt[p];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap, acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j] = acc[j] - off;
+      P = column_sum_f64<D>(reinterpret_cast<double*>(red), rg, cc, acc);
+    } else {
+#pragma unroll
+      for (int r = 0; r < G::RPT; ++r) {
+        const int i = r * G::NG + rg;
         const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -531,26 +648,24 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
           T[r][2 * p] = __fmul2_rn(make_float2(x.x, x.y), f2(gr[r]));
           T[r][2 * p + 1] = __fmul2_rn(make_float2(x.z, x.w), f2(gr[r]));
         }
-      }
 #pragma unroll
-      for (int p = 0; p < 8; ++p)
-        part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
-    }
-    {
-      const float P = column_sum<D>(red, rg, cc, part);
-      if (tid < D) {
-        const int j = tid;
-        const float beta = a.beta[(size_t)b * a.h_v + h];
-        if (PACKED) {
-          const float p = __fmul_rn(S.c()[j], P);
-          const float u = __fmul_rn(beta, __fsub_rn(S.v()[j], p));
-          wsh[j] = __fmul_rn(u, S.ic()[j]);
-        } else {
-          wsh[j] = __fmul_rn(beta, __fsub_rn(S.v()[j], P));
-        }
+        for (int p = 0; p < 8; ++p)
+          part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
       }
-      __syncthreads();
+      P = column_sum<D>(red, rg, cc, part);
     }
+    if (tid < D) {
+      const int j = tid;
+      const float beta = a.beta[(size_t)b * a.h_v + h];
+      if (PACKED) {
+        const float p = __fmul_rn(S.c()[j], P);
+        const float u = __fmul_rn(beta, __fsub_rn(S.v()[j], p));
+        wsh[j] = __fmul_rn(u, S.ic()[j]);
+      } else {
+        wsh[j] = __fmul_rn(beta, __fsub_rn(S.v()[j], P));
+      }
+    }
+    __syncthreads();
     float2 W[8];
     {
       const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
@@ -561,12 +676,17 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
         W[2 * p + 1] = make_float2(x.z, x.w);
       }
     }
-    // ---- pass B: delta update, partial S^T q
+    // ---- pass B: gate + delta update (one rounding), partial S^T q
 #pragma unroll
     for (int r = 0; r < G::RPT; ++r) {
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
+        if (PACKED) {
+          const float2 kw = __fmul2_rn(f2(kr[r]), W[p]);
+          T[r][p] = __ffma2_rn(T[r][p], f2(mr[r]), kw);
+        } else {
+          T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
+        }
         part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr[r])) : __ffma2_rn(T[r][p], f2(qr[r]), part[p]);
       }
     }

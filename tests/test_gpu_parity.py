@@ -29,7 +29,8 @@ def _cuda():
 
 def _report(name, stats, rollout):
     print(f"\n[{name}] steps={stats.steps} entries={stats.entries} flips={stats.flips} "
-          f"r_rows={stats.r_diff_rows} worst_o={stats.worst_o:.2e} rollout={rollout:.2e} {stats.notes}")
+          f"r_flips={stats.r_flips} max_diff={stats.max_code_diff} worst_o={stats.worst_o:.2e} "
+          f"rollout={rollout:.2e} {stats.notes}")
 
 
 def test_plumbing_config_full():
@@ -89,7 +90,8 @@ def test_edge_shapes_all_widths_and_pivots(d, gate_kind):
     B, h_v, h_k = 5, 6, 3
     bits, piv, col, phi = random_calib(rng, h_v, d, gate_kind, widths=(2, 4, 6, 8), pivot_p=0.15,
                                        phi_range=(0.3, 3.0))
-    cfg = synth.Config(99, "edge", gate_kind, B, h_v, h_k, d, 12, 64.0, (2, 4, 6, 8), 5, 0.0, 0.5, 1.0, 0, 0.0)
+    # the generator's own allocation is replaced by the random tables below
+    cfg = synth.Config(99, "edge", gate_kind, B, h_v, h_k, d, 12, 64.0, (8,), 8, 0.0, 0.5, 1.0, 0, 0.0)
     w = synth.Workload(cfg, seed=d)
     cal = w.calib()
     cal.unit_bits[...] = bits
