@@ -105,7 +105,7 @@ sq_status plan_step(sq_handle* h) {
   const bool packed = h->desc.fmt == SQ_FMT_PACKED;
   const uint32_t rec = packed ? (uint32_t)h->max_rec : (uint32_t)(4u * d * d);
   h->rec_cap = (uint32_t)round_up(rec, 128);
-  h->stage_bytes = (uint32_t)round_up(h->rec_cap + 31u * d, 128);
+  h->stage_bytes = (uint32_t)round_up(h->rec_cap + 31u * d + 32u, 128);  // + per-tile header
   const int NG = 32;  // row groups per CTA: 32 for every supported d
   const size_t red = (size_t)NG * d * (packed ? 8 : 4);  // fp64 column partials when packed
   int dev_max_smem = 0;

@@ -139,12 +139,13 @@ struct Geo {
   static constexpr int NT = 32 * NW;          // threads per CTA
   static constexpr int NG = NW * RPW;         // row groups (= rows per pass of the CTA)
   static constexpr int RPT = D / NG;          // rows per thread
-  static constexpr int AUX = 31 * D;          // aux bytes per stage (see stage layout)
+  static constexpr int AUX = 31 * D + 32;     // aux bytes per stage (see stage layout)
   static_assert(RPT >= 1 && RPT * NG == D, "bad geometry");
 };
 
 // Stage layout: [record: rec_cap][k f32 D][q f32 D][v f32 D][g f32 D]
 //               [c f32 D][ic f32 D][phi f32 D][row_off u16 D][row_code u8 D]
+//               [TileHdr 32 B]
 template <int D>
 struct Stage {
   uint8_t* base;
@@ -159,6 +160,19 @@ struct Stage {
   __device__ float* phi() const { return k() + 6 * D; }
   __device__ uint16_t* row_off() const { return reinterpret_cast<uint16_t*>(k() + 7 * D); }
   __device__ uint8_t* row_code() const { return reinterpret_cast<uint8_t*>(row_off() + D); }
+  __device__ struct TileHdr* hdr() const { return reinterpret_cast<struct TileHdr*>(row_code() + D); }
+};
+
+// Per-tile scalars the producing thread writes next to the stage's data
+// before the stage's mbarrier completes (so consumers never wait on global
+// memory for them).
+struct TileHdr {
+  uint8_t* dst;     // global address of the record (store target)
+  uint32_t bytes;   // record bytes
+  int32_t valid;    // 0: slot id out of range, nothing was loaded
+  float beta;
+  float g;          // the head's gate (GDN); unused for KDA
+  uint32_t pad[2];
 };
 
 // ------------------------------------------------------- code unpacking
@@ -449,14 +463,11 @@ __device__ __forceinline__ float column_sum(float* red, int rg, int cc, const fl
   return tot;
 }
 
-// fp64 column sums (same scheme as column_sum); returns the total rounded
-// once to fp32 for threads < D.
+// Total of the NG fp64 partials deposited per column in `red` (the caller
+// deposits, this syncs), rounded once to fp32; valid for threads < D.
 template <int D>
-__device__ __forceinline__ float column_sum_f64(double* red, int rg, int cc, const double (&part)[16]) {
+__device__ __forceinline__ float column_total_f64(const double* red) {
   using G = Geo<D>;
-  double2* dst = reinterpret_cast<double2*>(red + rg * D + 16 * cc);
-#pragma unroll
-  for (int p = 0; p < 8; ++p) dst[p] = make_double2(part[2 * p], part[2 * p + 1]);
   __syncthreads();
   float tot = 0.0f;
   if (threadIdx.x < D) {
@@ -478,38 +489,57 @@ __device__ __forceinline__ float column_sum_f64(double* red, int rg, int cc, con
 }
 
 // ================================================================ step kernel
+// Scalars of one tile, loaded by the producing thread one tile ahead of the
+// issue that needs them, so that their global-memory latency overlaps a
+// whole tile of compute.
+struct TileScalars {
+  int tile;
+  int b, h;
+  int slot;
+  uint32_t rec_off, rec_bytes;
+  float beta, g;
+};
+
 template <int D>
-__device__ __forceinline__ int tile_slot(const StepArgs& a, int b) {
-  return a.slots ? a.slots[b] : b;
+__device__ __forceinline__ TileScalars load_scalars(const StepArgs& a, int tile, int t1, bool packed) {
+  TileScalars x;
+  x.tile = tile;
+  if (tile >= t1) return x;
+  x.b = tile / a.h_v;
+  x.h = tile - x.b * a.h_v;
+  x.slot = a.slots ? a.slots[x.b] : x.b;
+  x.rec_off = packed ? a.t.rec_off[x.h] : 0u;
+  x.rec_bytes = packed ? a.t.rec_bytes[x.h] : 4u * D * D;
+  x.beta = a.beta[tile];
+  x.g = a.gate_kind == 0 ? a.g[tile] : 0.0f;
+  return x;
 }
 
 template <int D>
-__device__ __forceinline__ void issue_tile(const StepArgs& a, int tile, uint8_t* stage_base, uint64_t* bar,
-                                           bool packed) {
-  const int b = tile / a.h_v;
-  const int h = tile - b * a.h_v;
-  const int slot = tile_slot<D>(a, b);
-  if (slot < 0 || slot >= a.n_slots) {
+__device__ __forceinline__ void issue_tile(const StepArgs& a, const TileScalars& x, uint8_t* stage_base,
+                                           uint64_t* bar, bool packed) {
+  Stage<D> s{stage_base, a.rec_cap};
+  TileHdr* hd = s.hdr();
+  if (x.slot < 0 || x.slot >= a.n_slots) {
+    hd->valid = 0;
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
     return;
   }
-  Stage<D> s{stage_base, a.rec_cap};
+  const int b = x.b, h = x.h;
   const int hk = h / (a.h_v / a.h_k);
   const uint32_t vec = 4u * D;
   const bool kda = a.gate_kind != 0;
-  uint32_t rec_bytes;
-  const uint8_t* rec_src;
-  if (packed) {
-    rec_bytes = a.t.rec_bytes[h];
-    rec_src = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[h];
-  } else {
-    rec_bytes = 4u * D * D;
-    rec_src = a.pool + ((uint64_t)slot * a.h_v + h) * (uint64_t)(4u * D * D);
-  }
-  uint32_t tx = rec_bytes + 3 * vec + (kda ? vec : 0u);
+  uint8_t* rec_src = packed ? a.pool + (uint64_t)x.slot * a.slot_bytes + x.rec_off
+                            : a.pool + ((uint64_t)x.slot * a.h_v + h) * (uint64_t)(4u * D * D);
+  hd->dst = rec_src;
+  hd->bytes = x.rec_bytes;
+  hd->valid = 1;
+  hd->beta = x.beta;
+  hd->g = x.g;
+  uint32_t tx = x.rec_bytes + 3 * vec + (kda ? vec : 0u);
   if (packed) tx += 3 * vec + 2u * D + (uint32_t)D;
-  mbar_arrive_expect_tx(bar, tx);
-  bulk_g2s(s.rec(), rec_src, rec_bytes, bar);
+  mbar_arrive_expect_tx(bar, tx);  // release: the header stores above become visible with the phase
+  bulk_g2s(s.rec(), rec_src, x.rec_bytes, bar);
   bulk_g2s(s.k(), a.k + ((size_t)b * a.h_k + hk) * D, vec, bar);
   bulk_g2s(s.q(), a.q + ((size_t)b * a.h_k + hk) * D, vec, bar);
   bulk_g2s(s.v(), a.v + ((size_t)b * a.h_v + h) * D, vec, bar);
@@ -546,17 +576,20 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
   const int t1 = min(n_tiles, t0 + per);
   if (t0 >= t1) return;
 
+  TileScalars pre;  // thread 0: scalars of the next tile to issue
   if (tid == 0) {
     for (int s = 0; s < a.nstage; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     st_sh = 0;
     abort_sh = 0;
+    pre = load_scalars<D>(a, t0, t1, PACKED);
+    for (int s = 0; s < a.nstage && t0 + s < t1; ++s) {
+      const TileScalars cur = pre;
+      pre = load_scalars<D>(a, t0 + s + 1, t1, PACKED);
+      issue_tile<D>(a, cur, smem + (size_t)s * a.stage_bytes, &bars[s], PACKED);
+    }
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int s = 0; s < a.nstage && t0 + s < t1; ++s)
-      issue_tile<D>(a, t0 + s, smem + (size_t)s * a.stage_bytes, &bars[s], PACKED);
-  }
 
   uint32_t st = 0;
   for (int n = 0; t0 + n < t1; ++n) {
@@ -572,71 +605,84 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
 
     const int b = tile / a.h_v;
     const int h = tile - b * a.h_v;
-    const int slot = tile_slot<D>(a, b);
     float* o = a.o + ((size_t)b * a.h_v + h) * D;
-    if (slot < 0 || slot >= a.n_slots) {
+    const TileHdr hd = *S.hdr();
+    if (!hd.valid) {
       if (tid < D) o[tid] = 0.0f;
       st |= ST_SLOT;
       // nothing was loaded into this stage; refill it if there is work left
       __syncthreads();
-      if (tid == 0 && tile + a.nstage < t1) issue_tile<D>(a, tile + a.nstage, sbase, &bars[sidx], PACKED);
+      if (tid == 0 && tile + a.nstage < t1) {
+        const TileScalars cur = pre;
+        pre = load_scalars<D>(a, tile + a.nstage + 1, t1, PACKED);
+        issue_tile<D>(a, cur, sbase, &bars[sidx], PACKED);
+      }
       continue;
     }
 
     const float* ks = S.k();
     const float* qs = S.q();
     float kr[G::RPT], qr[G::RPT], gr[G::RPT];
-    const float gh = a.gate_kind == 0 ? a.g[(size_t)b * a.h_v + h] : 0.0f;
 #pragma unroll
     for (int r = 0; r < G::RPT; ++r) {
       const int i = r * G::NG + rg;
       kr[r] = ks[i];
       qr[r] = qs[i];
-      gr[r] = a.gate_kind == 0 ? gh : S.g()[i];
+      gr[r] = a.gate_kind == 0 ? hd.g : S.g()[i];
     }
 
     // ---- pass A: values, gate, column sum S^T k
     // packed: T holds the stored values V (codes or fp16) and mr the per-row
     // multiplier M (a_i = r_i g_i, or g_i for a pivot row); the column sum
-    // is accumulated in fp64 from the exact per-row factors (see unpack_hi).
+    // is accumulated in fp64 from the exact per-row factors (see unpack_hi),
+    // in two halves of 8 columns to keep the accumulators few.
     // fp32: T holds the gated state g_i S_ij and the column sum is fp32.
     float2 T[G::RPT][8];
     float mr[G::RPT];
     float2 part[8];
     float P;
     if (PACKED) {
-      double acc[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] = 0.0;
+      double kap[G::RPT];
       double off = 0.0;
 #pragma unroll
       for (int r = 0; r < G::RPT; ++r) {
         const int i = r * G::NG + rg;
         const uint8_t code = S.row_code()[i];
-        const uint8_t* row = S.rec() + S.row_off()[i];
-        double kap;
         if (code == ROW_PIVOT) {
           mr[r] = gr[r];
-          kap = (double)gr[r] * (double)kr[r];
+          kap[r] = (double)gr[r] * (double)kr[r];
         } else {
           const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
           mr[r] = __fmul_rn(R, gr[r]);
-          kap = (double)mr[r] * (double)kr[r] * (double)(1 << code);
-          off = off + 1.5 * kap;
+          kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << code);
+          off = off + 1.5 * kap[r];
         }
-        // unpack through temporaries: writing T[r] from inside the width
-        // switch would push the whole tile into local memory
-        float2 vt[8];
-        uint32_t xh[16];
-        unpack_hi(row, code, cc, vt, xh);
-#pragma unroll
-        for (int p = 0; p < 8; ++p) T[r][p] = vt[p];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap, acc[j]);
       }
+      double2* dst = reinterpret_cast<double2*>(reinterpret_cast<double*>(red) + rg * D + 16 * cc);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] = acc[j] - off;
-      P = column_sum_f64<D>(reinterpret_cast<double*>(red), rg, cc, acc);
+      for (int half = 0; half < 2; ++half) {
+        double acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+        for (int r = 0; r < G::RPT; ++r) {
+          const int i = r * G::NG + rg;
+          const uint8_t code = S.row_code()[i];
+          const uint8_t* row = S.rec() + S.row_off()[i];
+          // unpack through temporaries: writing T[r] from inside the width
+          // switch would push the whole tile into local memory
+          float2 vt[8];
+          uint32_t xh[16];
+          unpack_hi(row, code, cc, vt, xh);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) T[r][4 * half + p] = vt[4 * half + p];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[8 * half + j], 0), kap[r], acc[j]);
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) dst[4 * half + p] = make_double2(acc[2 * p] - off, acc[2 * p + 1] - off);
+      }
+      P = column_total_f64<D>(reinterpret_cast<double*>(red));
     } else {
 #pragma unroll
       for (int r = 0; r < G::RPT; ++r) {
@@ -656,13 +702,12 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     }
     if (tid < D) {
       const int j = tid;
-      const float beta = a.beta[(size_t)b * a.h_v + h];
       if (PACKED) {
         const float p = __fmul_rn(S.c()[j], P);
-        const float u = __fmul_rn(beta, __fsub_rn(S.v()[j], p));
+        const float u = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], p));
         wsh[j] = __fmul_rn(u, S.ic()[j]);
       } else {
-        wsh[j] = __fmul_rn(beta, __fsub_rn(S.v()[j], P));
+        wsh[j] = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
       }
     }
     __syncthreads();
@@ -714,19 +759,14 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      uint8_t* dst;
-      uint32_t bytes;
-      if (PACKED) {
-        dst = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[h];
-        bytes = a.t.rec_bytes[h];
-      } else {
-        dst = a.pool + ((uint64_t)slot * a.h_v + h) * (uint64_t)(4u * D * D);
-        bytes = 4u * D * D;
-      }
-      bulk_s2g(dst, S.rec(), bytes);
+      bulk_s2g(hd.dst, S.rec(), hd.bytes);
       bulk_commit();
       bulk_wait_read_all();
-      if (tile + a.nstage < t1) issue_tile<D>(a, tile + a.nstage, sbase, &bars[sidx], PACKED);
+      if (tile + a.nstage < t1) {
+        const TileScalars cur = pre;
+        pre = load_scalars<D>(a, tile + a.nstage + 1, t1, PACKED);
+        issue_tile<D>(a, cur, sbase, &bars[sidx], PACKED);
+      }
     }
   }
   if (st) atomicOr(&st_sh, st);
