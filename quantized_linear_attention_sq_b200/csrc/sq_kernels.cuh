@@ -204,36 +204,49 @@ __device__ __forceinline__ void unpack16(const uint32_t* w, float2 (&f)[8]) {
   }
 }
 
-// Field j of a 16-code chunk placed at bits [20-B, 20) of the word
-// 0x3FF00000. Read as the high word of a double (low word 0) this is
-// 1 + field * 2^-B exactly; read as a float it is 1.875 + field * 2^-(B+3).
-// One shift (or funnel shift) and one LOP3 per field give both.
+// Exponent E of the fp64 view of a field: the field sits at bits
+// [20-E, 20-E+B) of the word 0x3FF00000, so that, read as the high word of a
+// double (low word 0), the word is 1 + field * 2^-E exactly and, read as a
+// float, 1.875 + field * 2^-(E+3). 8-bit fields go to a byte boundary
+// (E = 12) so one byte permute places them; the others use E = B.
+template <int B>
+struct FieldPos {
+  static constexpr int E = B == 8 ? 12 : B;
+  static constexpr int POS = 20 - E;
+};
+
+// Field j of a 16-code chunk held in b/2 words, in place as described above.
 template <int B>
 __device__ __forceinline__ uint32_t field_hi(const uint32_t* w, int j) {
-  constexpr int POS = 20 - B;
-  constexpr uint32_t MASK = ((1u << B) - 1u) << POS;
-  const int bit = B * j;
-  const int wi = bit >> 5;
-  const int sh = bit & 31;
-  uint32_t x;
-  if (sh + B <= 32)
-    x = sh >= POS ? (w[wi] >> (sh - POS)) : (w[wi] << (POS - sh));
-  else
-    x = __funnelshift_r(w[wi], w[wi + 1], sh - POS);  // a straddling field always has sh > POS
-  return 0x3FF00000u | (x & MASK);
+  constexpr int POS = FieldPos<B>::POS;
+  if constexpr (B == 8) {
+    return __byte_perm(w[j >> 2], 0x3FF00000u, 0x7604u | ((uint32_t)(j & 3) << 4));
+  } else {
+    constexpr uint32_t MASK = ((1u << B) - 1u) << POS;
+    const int bit = B * j;
+    const int wi = bit >> 5;
+    const int sh = bit & 31;
+    uint32_t x;
+    if (sh + B <= 32)
+      x = sh >= POS ? (w[wi] >> (sh - POS)) : (w[wi] << (POS - sh));
+    else
+      x = __funnelshift_r(w[wi], w[wi + 1], sh - POS);  // a straddling field always has sh > POS
+    return 0x3FF00000u | (x & MASK);
+  }
 }
 
 // Pass-A unpack of one quantized 16-code chunk: the codes q as floats (exact)
-// and the high words of the doubles 1 + field * 2^-B that feed the fp64
-// column sum (with the per-row factor 2^B a k, minus 1.5 2^B a k per row,
-// they give q a k exactly up to fp64 rounding).
+// and the high words of the doubles 1 + field * 2^-E that feed the fp64
+// column sum (with the per-row factor 2^E a k, minus (1 + 2^(B-1-E)) 2^E a k
+// per row, they give q a k up to fp64 rounding).
 template <int B>
 __device__ __forceinline__ void unpack_q_hi(const uint8_t* row, int cc, float2 (&V)[8], uint32_t (&xh)[16]) {
   const uint32_t* src = reinterpret_cast<const uint32_t*>(row + 2 * B * cc);
   uint32_t w[B / 2];
 #pragma unroll
   for (int i = 0; i < B / 2; ++i) w[i] = src[i];
-  const float S = (float)(1 << (B + 3));
+  constexpr int E = FieldPos<B>::E;
+  const float S = (float)(1 << (E + 3));
   const float C = 1.875f * S + (float)(1 << (B - 1));
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
@@ -270,24 +283,49 @@ __device__ __forceinline__ void unpack_hi(const uint8_t* row, uint8_t code, int 
   }
 }
 
-// Pack 16 magic-number floats (2^23 + field) into b/2 words.
+// Constant part of packed word `wi` when every fb[j] = 0x4B000000 + field_j
+// is shifted into place (see pack16).
+template <int B>
+__host__ __device__ constexpr uint32_t pack_const(int wi) {
+  uint32_t c = 0;
+  for (int j = 0; j < 16; ++j) {
+    const int lo = B * j - 32 * wi;
+    if (lo >= 32 || lo + B <= 0) continue;
+    c += lo >= 0 ? (0x4B000000u << lo) : (0x4B000000u >> (-lo));
+  }
+  return c;
+}
+
+// Pack 16 magic-number floats fb[j] = bits(2^23 + field_j) into b/2 words.
+// 8-bit: byte permutes. Otherwise: the fields occupy disjoint bits and the
+// constant 0x4B000000 is a multiple of 2^24 (so shifting it right by less
+// than 24 never mixes with a field), hence each word is the sum of the
+// shifted fb[j] minus the same sum of shifted constants (mod 2^32): one
+// multiply-add per field.
 template <int B>
 __device__ __forceinline__ void pack16(const uint32_t (&fb)[16], uint32_t* w) {
-  constexpr uint32_t mask = (1u << B) - 1u;
+  if constexpr (B == 8) {
 #pragma unroll
-  for (int wi = 0; wi < B / 2; ++wi) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int lo = B * j - 32 * wi;
-      if (lo >= 32 || lo + B <= 0) continue;
-      const uint32_t f = fb[j] & mask;
-      if (lo >= 0)
-        word |= f << lo;
-      else
-        word |= f >> (-lo);
+    for (int wi = 0; wi < 4; ++wi) {
+      const uint32_t lo = __byte_perm(fb[4 * wi], fb[4 * wi + 1], 0x0040);
+      const uint32_t hi = __byte_perm(fb[4 * wi + 2], fb[4 * wi + 3], 0x0040);
+      w[wi] = __byte_perm(lo, hi, 0x5410);
     }
-    w[wi] = word;
+  } else {
+#pragma unroll
+    for (int wi = 0; wi < B / 2; ++wi) {
+      uint32_t acc = 0u - pack_const<B>(wi);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int lo = B * j - 32 * wi;
+        if (lo >= 32 || lo + B <= 0) continue;
+        if (lo >= 0)
+          acc += fb[j] * (1u << lo);
+        else
+          acc += fb[j] >> (-lo);
+      }
+      w[wi] = acc;
+    }
   }
 }
 
@@ -382,110 +420,149 @@ __device__ __forceinline__ uint32_t store_row_pivot(uint8_t* row, int cc, const 
   return st;
 }
 
-// Steps 7-10 for the RPT rows a thread holds: row maxima across the LPR lanes
-// of each row, row scales, codes; writes the record in shared memory.
-// Returns the status bits this thread raised.
+// Requantization of the RPT rows a thread holds: row maxima across the LPR
+// lanes of each row, one row scale per row (computed by one lane of the row
+// and handed to the others by shuffle), codes; writes the record in shared
+// memory. `finite`: the tile's inputs were all finite, so no T' is NaN and
+// the plain maximum equals the NaN-propagating one. Returns status bits.
 template <int D>
 __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
-                                                 const float* phi, int rg, int cc, float2 (&T)[Geo<D>::RPT][8]) {
+                                                 const float* phi, int rg, int cc, bool finite,
+                                                 float2 (&T)[Geo<D>::RPT][8]) {
   using G = Geo<D>;
   uint32_t st = 0;
+  float m[G::RPT];
 #pragma unroll
   for (int r = 0; r < G::RPT; ++r) {
+    float x = 0.0f;
+    if (finite) {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) x = fmaxf(x, fmaxf(fabsf(T[r][p].x), fabsf(T[r][p].y)));
+#pragma unroll
+      for (int s = 1; s < G::LPR; s <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, s));
+    } else {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) x = fmax_nan(x, fmax_nan(fabsf(T[r][p].x), fabsf(T[r][p].y)));
+#pragma unroll
+      for (int s = 1; s < G::LPR; s <<= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, s));
+    }
+    m[r] = x;
+  }
+  // lane cc of a row group computes the scale of row slot cc % RPT
+  const int mine = cc % G::RPT;
+  float mm = m[0];
+#pragma unroll
+  for (int r = 1; r < G::RPT; ++r) mm = mine == r ? m[r] : mm;
+  const int im = mine * G::NG + rg;
+  const int cm = row_code[im];
+  float ir_m = 0.0f;
+  uint16_t rbits = 0x3C00;  // pivot rows keep fp16 1.0 in their scale slot
+  if (cm != ROW_PIVOT) {
+    if (mm != mm) {
+      rbits = 0;
+      st |= ST_NAN;
+    } else {
+      const float qm = (float)((1 << (cm - 1)) - 1);
+      const float s = __fdiv_rn(__fmul_rn(phi[im], mm), qm);
+      __half rh;
+      if (s > 65504.0f) {
+        rh = __ushort_as_half((unsigned short)0x7BFF);
+        st |= ST_SAT;
+      } else {
+        rh = __float2half_ru(s);
+      }
+      const float R = __half2float(rh);
+      ir_m = (R == 0.0f) ? 0.0f : __frcp_rn(R);
+      rbits = __half_as_ushort(rh);
+    }
+  }
+  if (cc < G::RPT) reinterpret_cast<uint16_t*>(rec)[im] = rbits;
+  const int lane = threadIdx.x & 31;
+  const int base = lane - cc;
+#pragma unroll
+  for (int r = 0; r < G::RPT; ++r) {
+    const float ir = __shfl_sync(0xffffffffu, ir_m, base + r);
     const int i = r * G::NG + rg;
     const uint8_t code = row_code[i];
     uint8_t* row = rec + row_off[i];
-    float m = 0.0f;
-#pragma unroll
-    for (int p = 0; p < 8; ++p) m = fmax_nan(m, fmax_nan(fabsf(T[r][p].x), fabsf(T[r][p].y)));
-#pragma unroll
-    for (int s = 1; s < G::LPR; s <<= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, s));
     if (code == ROW_PIVOT) {
       st |= store_row_pivot(row, cc, T[r]);
-      if (cc == 0) reinterpret_cast<uint16_t*>(rec)[i] = 0x3C00;
-      continue;
-    }
-    const int B = code;
-    if (m != m) {  // a NaN in the row: scale 0, all codes 0
-      st |= ST_NAN;
-      store_row_zero(row, B, cc);
-      if (cc == 0) reinterpret_cast<uint16_t*>(rec)[i] = 0;
-      continue;
-    }
-    const float qm = (float)((1 << (B - 1)) - 1);
-    const float s = __fdiv_rn(__fmul_rn(phi[i], m), qm);
-    __half rh;
-    if (s > 65504.0f) {
-      rh = __ushort_as_half((unsigned short)0x7BFF);
-      st |= ST_SAT;
+    } else if (m[r] != m[r]) {  // a NaN in the row: scale 0, all codes 0
+      store_row_zero(row, code, cc);
     } else {
-      rh = __float2half_ru(s);
-    }
-    const float R = __half2float(rh);
-    const float ir = (R == 0.0f) ? 0.0f : __frcp_rn(R);
-    if (cc == 0) reinterpret_cast<uint16_t*>(rec)[i] = __half_as_ushort(rh);
-    switch (B) {
-      case 8: store_row_q<8>(row, cc, ir, T[r]); break;
-      case 6: store_row_q<6>(row, cc, ir, T[r]); break;
-      case 4: store_row_q<4>(row, cc, ir, T[r]); break;
-      default: store_row_q<2>(row, cc, ir, T[r]); break;
+      switch (code) {
+        case 8: store_row_q<8>(row, cc, ir, T[r]); break;
+        case 6: store_row_q<6>(row, cc, ir, T[r]); break;
+        case 4: store_row_q<4>(row, cc, ir, T[r]); break;
+        default: store_row_q<2>(row, cc, ir, T[r]); break;
+      }
     }
   }
   return st;
 }
 
-// Column sums: every thread deposits its 16 partial sums; the first D
-// threads add the NG partials of one column. Returns the column total for
-// threads < D (undefined otherwise). Caller syncs before reusing `red`.
+// Column sums. Every thread deposits its 16 partials for its row group;
+// a thread's chunks are stored rotated by its column block (XOR swizzle) so
+// the eight lanes of a row write eight different bank groups. Then two
+// adjacent threads own one column (thread 2j and 2j+1 each add half of the
+// row groups) and combine with one shuffle. Returns the column total in
+// every thread of the pair; column = threadIdx.x >> 1. The caller syncs
+// before reusing `red`.
 template <int D>
 __device__ __forceinline__ float column_sum(float* red, int rg, int cc, const float2 (&part)[8]) {
   using G = Geo<D>;
-  float4* dst = reinterpret_cast<float4*>(red + rg * D + 16 * cc);
+  static_assert(G::NT == 2 * D, "two threads per column");
+  const int sw = (cc >> 1) & 3;
 #pragma unroll
-  for (int p = 0; p < 4; ++p) dst[p] = make_float4(part[2 * p].x, part[2 * p].y, part[2 * p + 1].x, part[2 * p + 1].y);
+  for (int p = 0; p < 4; ++p)
+    *reinterpret_cast<float4*>(red + rg * D + 16 * cc + 4 * (p ^ sw)) =
+        make_float4(part[2 * p].x, part[2 * p].y, part[2 * p + 1].x, part[2 * p + 1].y);
   __syncthreads();
-  float tot = 0.0f;
-  if (threadIdx.x < D) {
-    const int j = threadIdx.x;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int g = 0;
+  const int j = threadIdx.x >> 1;
+  const int hh = threadIdx.x & 1;
+  const int cj = j >> 4, e = j & 15;
+  const int off = 16 * cj + 4 * ((e >> 2) ^ ((cj >> 1) & 3)) + (e & 3);
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (; g + 3 < G::NG; g += 4) {
-      a0 = __fadd_rn(a0, red[(g + 0) * D + j]);
-      a1 = __fadd_rn(a1, red[(g + 1) * D + j]);
-      a2 = __fadd_rn(a2, red[(g + 2) * D + j]);
-      a3 = __fadd_rn(a3, red[(g + 3) * D + j]);
-    }
-#pragma unroll
-    for (; g < G::NG; ++g) a0 = __fadd_rn(a0, red[g * D + j]);
-    tot = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+  for (int g = 0; g < G::NG / 2; g += 2) {
+    a0 = __fadd_rn(a0, red[(hh * (G::NG / 2) + g) * D + off]);
+    a1 = __fadd_rn(a1, red[(hh * (G::NG / 2) + g + 1) * D + off]);
   }
-  return tot;
+  const float a = __fadd_rn(a0, a1);
+  return __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
 }
 
-// Total of the NG fp64 partials deposited per column in `red` (the caller
-// deposits, this syncs), rounded once to fp32; valid for threads < D.
+// fp64 deposit of the 16 pass-A partials (same swizzle idea, 16-byte chunks
+// of two doubles rotated by cc).
+template <int D>
+__device__ __forceinline__ void deposit_f64(double* red, int rg, int cc, int half, const double (&acc)[8],
+                                            double off) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int chunk = 4 * half + p;
+    *reinterpret_cast<double2*>(red + rg * D + 16 * cc + 2 * (chunk ^ (cc & 7))) =
+        make_double2(acc[2 * p] - off, acc[2 * p + 1] - off);
+  }
+}
+
+// Column total of the fp64 partials, rounded once to fp32 (two threads per
+// column as in column_sum; column = threadIdx.x >> 1). Syncs first.
 template <int D>
 __device__ __forceinline__ float column_total_f64(const double* red) {
   using G = Geo<D>;
   __syncthreads();
-  float tot = 0.0f;
-  if (threadIdx.x < D) {
-    const int j = threadIdx.x;
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-    int g = 0;
+  const int j = threadIdx.x >> 1;
+  const int hh = threadIdx.x & 1;
+  const int cj = j >> 4, e = j & 15;
+  const int off = 16 * cj + 2 * ((e >> 1) ^ (cj & 7)) + (e & 1);
+  double a0 = 0.0, a1 = 0.0;
 #pragma unroll
-    for (; g + 3 < G::NG; g += 4) {
-      a0 += red[(g + 0) * D + j];
-      a1 += red[(g + 1) * D + j];
-      a2 += red[(g + 2) * D + j];
-      a3 += red[(g + 3) * D + j];
-    }
-#pragma unroll
-    for (; g < G::NG; ++g) a0 += red[g * D + j];
-    tot = __double2float_rn((a0 + a1) + (a2 + a3));
+  for (int g = 0; g < G::NG / 2; g += 2) {
+    a0 += red[(hh * (G::NG / 2) + g) * D + off];
+    a1 += red[(hh * (G::NG / 2) + g + 1) * D + off];
   }
-  return tot;
+  const double a = a0 + a1;
+  return __double2float_rn(a + __shfl_xor_sync(0xffffffffu, a, 1));
 }
 
 // ================================================================ step kernel
@@ -562,6 +639,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
   __shared__ __align__(16) float wsh[D];
   __shared__ uint32_t st_sh;
   __shared__ int abort_sh;
+  __shared__ int nf_sh;  // the current tile saw a non-finite input
   float* red = reinterpret_cast<float*>(smem + (size_t)a.nstage * a.stage_bytes);
 
   const int tid = threadIdx.x;
@@ -582,6 +660,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     fence_mbar_init();
     st_sh = 0;
     abort_sh = 0;
+    nf_sh = 0;
     pre = load_scalars<D>(a, t0, t1, PACKED);
     for (int s = 0; s < a.nstage && t0 + s < t1; ++s) {
       const TileScalars cur = pre;
@@ -608,7 +687,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     float* o = a.o + ((size_t)b * a.h_v + h) * D;
     const TileHdr hd = *S.hdr();
     if (!hd.valid) {
-      if (tid < D) o[tid] = 0.0f;
+      if (tid < D) o[tid] = 0.0f;  // (nf_sh stays 0: nothing was computed)
       st |= ST_SLOT;
       // nothing was loaded into this stage; refill it if there is work left
       __syncthreads();
@@ -644,6 +723,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     if (PACKED) {
       double kap[G::RPT];
       double off = 0.0;
+      bool bad = false;
 #pragma unroll
       for (int r = 0; r < G::RPT; ++r) {
         const int i = r * G::NG + rg;
@@ -654,11 +734,13 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
         } else {
           const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
           mr[r] = __fmul_rn(R, gr[r]);
-          kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << code);
-          off = off + 1.5 * kap[r];
+          const int E = code == 8 ? 12 : code;  // FieldPos<code>::E
+          kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << E);
+          off = off + (1.0 + (double)(1 << (code - 1)) / (double)(1 << E)) * kap[r];
         }
+        bad |= !isfinite(mr[r]) || !isfinite(kr[r]);
       }
-      double2* dst = reinterpret_cast<double2*>(reinterpret_cast<double*>(red) + rg * D + 16 * cc);
+      double* red64 = reinterpret_cast<double*>(red);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         double acc[8];
@@ -676,13 +758,17 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
           unpack_hi(row, code, cc, vt, xh);
 #pragma unroll
           for (int p = 0; p < 4; ++p) T[r][4 * half + p] = vt[4 * half + p];
+          if (code == ROW_PIVOT) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) bad |= !isfinite(vt[4 * half + p].x) || !isfinite(vt[4 * half + p].y);
+          }
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[8 * half + j], 0), kap[r], acc[j]);
         }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) dst[4 * half + p] = make_double2(acc[2 * p] - off, acc[2 * p + 1] - off);
+        deposit_f64<D>(red64, rg, cc, half, acc, off);
       }
-      P = column_total_f64<D>(reinterpret_cast<double*>(red));
+      if (bad) nf_sh = 1;
+      P = column_total_f64<D>(red64);
     } else {
 #pragma unroll
       for (int r = 0; r < G::RPT; ++r) {
@@ -700,17 +786,21 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
       }
       P = column_sum<D>(red, rg, cc, part);
     }
-    if (tid < D) {
-      const int j = tid;
+    if ((tid & 1) == 0) {
+      const int j = tid >> 1;
+      float wj;
       if (PACKED) {
         const float p = __fmul_rn(S.c()[j], P);
         const float u = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], p));
-        wsh[j] = __fmul_rn(u, S.ic()[j]);
+        wj = __fmul_rn(u, S.ic()[j]);
+        if (!isfinite(wj)) nf_sh = 1;
       } else {
-        wsh[j] = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
+        wj = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
       }
+      wsh[j] = wj;
     }
     __syncthreads();
+    const bool finite = nf_sh == 0;
     float2 W[8];
     {
       const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
@@ -737,15 +827,16 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     }
     {
       const float O = column_sum<D>(red, rg, cc, part);
-      if (tid < D) {
-        const float oj = PACKED ? __fmul_rn(S.c()[tid], O) : O;
+      if ((tid & 1) == 0) {
+        const int j = tid >> 1;
+        const float oj = PACKED ? __fmul_rn(S.c()[j], O) : O;
         if (oj != oj) st |= ST_NAN;
-        o[tid] = oj;
+        o[j] = oj;
       }
     }
     // ---- requantize (or store fp32) into the stage record, in place
     if (PACKED) {
-      st |= requant_rows<D>(S.rec(), S.row_off(), S.row_code(), S.phi(), rg, cc, T);
+      st |= requant_rows<D>(S.rec(), S.row_off(), S.row_code(), S.phi(), rg, cc, finite, T);
     } else {
 #pragma unroll
       for (int r = 0; r < G::RPT; ++r) {
@@ -759,6 +850,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
+      nf_sh = 0;  // every read of this tile's flag happened before the barrier above
       bulk_s2g(hd.dst, S.rec(), hd.bytes);
       bulk_commit();
       bulk_wait_read_all();
@@ -839,7 +931,7 @@ __global__ void __launch_bounds__(Geo<D>::NT) k_quantize(const QuantArgs a) {
     }
   }
   __syncthreads();
-  uint32_t st = requant_rows<D>(rec, row_off, row_code, phi, rg, cc, T);
+  uint32_t st = requant_rows<D>(rec, row_off, row_code, phi, rg, cc, false, T);
   __syncthreads();
   uint8_t* dst = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[h];
   for (uint32_t x = tid * 16; x < rb; x += G::NT * 16) *reinterpret_cast<uint4*>(dst + x) = *reinterpret_cast<uint4*>(rec + x);
