@@ -246,7 +246,8 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   size_t o_phi = round_up(o_icol + 4 * nhd, 16);
   size_t o_row_off = round_up(o_phi + 4 * nhd, 16);
   size_t o_row_code = round_up(o_row_off + 2 * nhd, 16);
-  size_t o_status = round_up(o_row_code + nhd, 16);
+  size_t o_head_kind = round_up(o_row_code + nhd, 16);
+  size_t o_status = round_up(o_head_kind + hv, 16);
   size_t total = round_up(o_status + 16, 256);
   std::vector<uint8_t> host(total, 0);
   memcpy(host.data() + o_rec_off, h->rec_off.data(), 4 * hv);
@@ -262,6 +263,12 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   }
   memcpy(host.data() + o_row_off, h->row_off.data(), 2 * nhd);
   memcpy(host.data() + o_row_code, h->row_code.data(), nhd);
+  for (int hh = 0; hh < hv; ++hh) {  // width shared by every row of the head, else 0
+    uint8_t k = packed ? h->row_code[(size_t)hh * d] : 0;
+    for (int i = 1; i < d && k; ++i)
+      if (h->row_code[(size_t)hh * d + i] != k) k = 0;
+    host[o_head_kind + hh] = k;
+  }
   e = cudaMalloc(&h->dev_block, total);
   if (e != cudaSuccess) {
     delete h;
@@ -282,6 +289,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   h->tables.phi = reinterpret_cast<const float*>(base + o_phi);
   h->tables.row_off = reinterpret_cast<const uint16_t*>(base + o_row_off);
   h->tables.row_code = reinterpret_cast<const uint8_t*>(base + o_row_code);
+  h->tables.head_kind = reinterpret_cast<const uint8_t*>(base + o_head_kind);
   h->tables.status = reinterpret_cast<uint32_t*>(base + o_status);
   s = plan_step(h);
   if (s != SQ_OK) {

@@ -45,6 +45,7 @@ struct Tables {
   const float* col;           // [h_v*d] c_j
   const float* icol;          // [h_v*d] fl(1 / c_j)
   const float* phi;           // [h_v*d] phi_i
+  const uint8_t* head_kind;   // [h_v] width shared by all rows of the head (ROW_PIVOT: all pivot), 0: mixed
   uint32_t* status;           // device status word
 };
 
@@ -172,7 +173,8 @@ struct TileHdr {
   int32_t valid;    // 0: slot id out of range, nothing was loaded
   float beta;
   float g;          // the head's gate (GDN); unused for KDA
-  uint32_t pad[2];
+  int32_t kind;     // width shared by every row of the head (ROW_PIVOT: all pivot), 0: mixed
+  uint32_t pad;
 };
 
 // ------------------------------------------------------- code unpacking
@@ -390,10 +392,10 @@ __device__ __forceinline__ void store_row_q(uint8_t* row, int cc, float ir, cons
 }
 
 __device__ __forceinline__ void store_row_zero(uint8_t* row, int B, int cc) {
-  // all codes 0: every field is 2^(b-1)
+  // all codes 0: every field is 2^(b-1) (given to pack16 in its 2^23 + field form)
   uint32_t fb[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) fb[j] = 1u << (B - 1);
+  for (int j = 0; j < 16; ++j) fb[j] = 0x4B000000u | (1u << (B - 1));
   uint32_t* dst = reinterpret_cast<uint32_t*>(row + 2 * B * cc);
   switch (B) {
     case 8: { uint32_t w[4]; pack16<8>(fb, w); for (int i = 0; i < 4; ++i) dst[i] = w[i]; } break;
@@ -420,16 +422,30 @@ __device__ __forceinline__ uint32_t store_row_pivot(uint8_t* row, int cc, const 
   return st;
 }
 
+// Byte offset of key row i inside a head record: from the per-head table,
+// or, when every row of the head has width KC (KC = ROW_PIVOT for an
+// all-pivot head), from the closed form 2d + i * row_bytes.
+template <int D, int KC>
+__device__ __forceinline__ uint32_t row_offset(const uint16_t* row_off, int i) {
+  if constexpr (KC == 0) {
+    return row_off[i];
+  } else {
+    constexpr uint32_t rb = KC == ROW_PIVOT ? 2u * D : (uint32_t)(D * KC / 8);
+    return 2u * D + (uint32_t)i * rb;
+  }
+}
+
 // Requantization of the RPT rows a thread holds: row maxima across the LPR
 // lanes of each row, one row scale per row (computed by one lane of the row
 // and handed to the others by shuffle), codes; writes the record in shared
 // memory. `finite`: the tile's inputs were all finite, so no T' is NaN and
 // the plain maximum equals the NaN-propagating one. Returns status bits.
-template <int D>
+template <int D, int KC>
 __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
                                                  const float* phi, int rg, int cc, bool finite,
                                                  float2 (&T)[Geo<D>::RPT][8]) {
   using G = Geo<D>;
+  (void)row_off;
   uint32_t st = 0;
   float m[G::RPT];
 #pragma unroll
@@ -454,7 +470,7 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
 #pragma unroll
   for (int r = 1; r < G::RPT; ++r) mm = mine == r ? m[r] : mm;
   const int im = mine * G::NG + rg;
-  const int cm = row_code[im];
+  const int cm = KC ? KC : row_code[im];
   float ir_m = 0.0f;
   uint16_t rbits = 0x3C00;  // pivot rows keep fp16 1.0 in their scale slot
   if (cm != ROW_PIVOT) {
@@ -483,8 +499,8 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
   for (int r = 0; r < G::RPT; ++r) {
     const float ir = __shfl_sync(0xffffffffu, ir_m, base + r);
     const int i = r * G::NG + rg;
-    const uint8_t code = row_code[i];
-    uint8_t* row = rec + row_off[i];
+    const int code = KC ? KC : row_code[i];
+    uint8_t* row = rec + row_offset<D, KC>(row_off, i);
     if (code == ROW_PIVOT) {
       st |= store_row_pivot(row, cc, T[r]);
     } else if (m[r] != m[r]) {  // a NaN in the row: scale 0, all codes 0
@@ -575,6 +591,7 @@ struct TileScalars {
   int slot;
   uint32_t rec_off, rec_bytes;
   float beta, g;
+  int kind;
 };
 
 template <int D>
@@ -589,6 +606,7 @@ __device__ __forceinline__ TileScalars load_scalars(const StepArgs& a, int tile,
   x.rec_bytes = packed ? a.t.rec_bytes[x.h] : 4u * D * D;
   x.beta = a.beta[tile];
   x.g = a.gate_kind == 0 ? a.g[tile] : 0.0f;
+  x.kind = packed ? a.t.head_kind[x.h] : 0;
   return x;
 }
 
@@ -613,6 +631,7 @@ __device__ __forceinline__ void issue_tile(const StepArgs& a, const TileScalars&
   hd->valid = 1;
   hd->beta = x.beta;
   hd->g = x.g;
+  hd->kind = x.kind;
   uint32_t tx = x.rec_bytes + 3 * vec + (kda ? vec : 0u);
   if (packed) tx += 3 * vec + 2u * D + (uint32_t)D;
   mbar_arrive_expect_tx(bar, tx);  // release: the header stores above become visible with the phase
@@ -627,6 +646,166 @@ __device__ __forceinline__ void issue_tile(const StepArgs& a, const TileScalars&
     bulk_g2s(s.phi(), a.t.phi + (size_t)h * D, vec, bar);
     bulk_g2s(s.row_off(), a.t.row_off + (size_t)h * D, 2u * D, bar);
     bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
+  }
+}
+
+// The compute of one tile, from the stage in shared memory to the updated
+// record written back into the stage and o written to global memory. KC is
+// the width shared by every row of the head (ROW_PIVOT for an all-pivot
+// head), known at compile time, or 0 for heads whose rows differ (KDA):
+// with KC != 0 every per-row width switch folds away.
+template <int D, bool PACKED, int KC>
+__device__ __forceinline__ void tile_body(const StepArgs& a, const Stage<D>& S, const TileHdr& hd, float* red,
+                                          float* wsh, int* nf_sh, float* o, int rg, int cc, uint32_t& st) {
+  using G = Geo<D>;
+  const int tid = threadIdx.x;
+  const float* ks = S.k();
+  const float* qs = S.q();
+  float kr[G::RPT], qr[G::RPT], gr[G::RPT];
+#pragma unroll
+  for (int r = 0; r < G::RPT; ++r) {
+    const int i = r * G::NG + rg;
+    kr[r] = ks[i];
+    qr[r] = qs[i];
+    gr[r] = a.gate_kind == 0 ? hd.g : S.g()[i];
+  }
+
+  // ---- pass A: values, gate, column sum S^T k
+  // packed: T holds the stored values V (codes or fp16) and mr the per-row
+  // multiplier M (a_i = r_i g_i, or g_i for a pivot row); the column sum
+  // is accumulated in fp64 from the exact per-row factors (see unpack_hi),
+  // in two halves of 8 columns to keep the accumulators few.
+  // fp32: T holds the gated state g_i S_ij and the column sum is fp32.
+  float2 T[G::RPT][8];
+  float mr[G::RPT];
+  float2 part[8];
+  float P;
+  if (PACKED) {
+    double kap[G::RPT];
+    double off = 0.0;
+    bool bad = false;
+#pragma unroll
+    for (int r = 0; r < G::RPT; ++r) {
+      const int i = r * G::NG + rg;
+      const int code = KC ? KC : S.row_code()[i];
+      if (code == ROW_PIVOT) {
+        mr[r] = gr[r];
+        kap[r] = (double)gr[r] * (double)kr[r];
+      } else {
+        const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
+        mr[r] = __fmul_rn(R, gr[r]);
+        const int E = code == 8 ? 12 : code;  // FieldPos<code>::E
+        kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << E);
+        off = off + (1.0 + (double)(1 << (code - 1)) / (double)(1 << E)) * kap[r];
+      }
+      bad |= !isfinite(mr[r]) || !isfinite(kr[r]);
+    }
+    double* red64 = reinterpret_cast<double*>(red);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      double acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+      for (int r = 0; r < G::RPT; ++r) {
+        const int i = r * G::NG + rg;
+        const int code = KC ? KC : S.row_code()[i];
+        const uint8_t* row = S.rec() + row_offset<D, KC>(S.row_off(), i);
+        // unpack through temporaries: writing T[r] from inside the width
+        // switch would push the whole tile into local memory
+        float2 vt[8];
+        uint32_t xh[16];
+        unpack_hi(row, code, cc, vt, xh);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) T[r][4 * half + p] = vt[4 * half + p];
+        if (code == ROW_PIVOT) {
+#pragma unroll
+          for (int p = 0; p < 4; ++p) bad |= !isfinite(vt[4 * half + p].x) || !isfinite(vt[4 * half + p].y);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[8 * half + j], 0), kap[r], acc[j]);
+      }
+      deposit_f64<D>(red64, rg, cc, half, acc, off);
+    }
+    if (bad) *nf_sh = 1;
+    P = column_total_f64<D>(red64);
+  } else {
+#pragma unroll
+    for (int r = 0; r < G::RPT; ++r) {
+      const int i = r * G::NG + rg;
+      const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        float4 x = src[p];
+        T[r][2 * p] = __fmul2_rn(make_float2(x.x, x.y), f2(gr[r]));
+        T[r][2 * p + 1] = __fmul2_rn(make_float2(x.z, x.w), f2(gr[r]));
+      }
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
+    }
+    P = column_sum<D>(red, rg, cc, part);
+  }
+  if ((tid & 1) == 0) {
+    const int j = tid >> 1;
+    float wj;
+    if (PACKED) {
+      const float p = __fmul_rn(S.c()[j], P);
+      const float u = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], p));
+      wj = __fmul_rn(u, S.ic()[j]);
+      if (!isfinite(wj)) *nf_sh = 1;
+    } else {
+      wj = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
+    }
+    wsh[j] = wj;
+  }
+  __syncthreads();
+  const bool finite = *nf_sh == 0;
+  float2 W[8];
+  {
+    const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      float4 x = wsrc[p];
+      W[2 * p] = make_float2(x.x, x.y);
+      W[2 * p + 1] = make_float2(x.z, x.w);
+    }
+  }
+  // ---- pass B: gate + delta update (one rounding), partial S^T q
+#pragma unroll
+  for (int r = 0; r < G::RPT; ++r) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if (PACKED) {
+        const float2 kw = __fmul2_rn(f2(kr[r]), W[p]);
+        T[r][p] = __ffma2_rn(T[r][p], f2(mr[r]), kw);
+      } else {
+        T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
+      }
+      part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr[r])) : __ffma2_rn(T[r][p], f2(qr[r]), part[p]);
+    }
+  }
+  {
+    const float O = column_sum<D>(red, rg, cc, part);
+    if ((tid & 1) == 0) {
+      const int j = tid >> 1;
+      const float oj = PACKED ? __fmul_rn(S.c()[j], O) : O;
+      if (oj != oj) st |= ST_NAN;
+      o[j] = oj;
+    }
+  }
+  // ---- requantize (or store fp32) into the stage record, in place
+  if (PACKED) {
+    st |= requant_rows<D, KC>(S.rec(), S.row_off(), S.row_code(), S.phi(), rg, cc, finite, T);
+  } else {
+#pragma unroll
+    for (int r = 0; r < G::RPT; ++r) {
+      const int i = r * G::NG + rg;
+      float4* dst = reinterpret_cast<float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        dst[p] = make_float4(T[r][2 * p].x, T[r][2 * p].y, T[r][2 * p + 1].x, T[r][2 * p + 1].y);
+    }
   }
 }
 
@@ -699,153 +878,13 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
       continue;
     }
 
-    const float* ks = S.k();
-    const float* qs = S.q();
-    float kr[G::RPT], qr[G::RPT], gr[G::RPT];
-#pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const int i = r * G::NG + rg;
-      kr[r] = ks[i];
-      qr[r] = qs[i];
-      gr[r] = a.gate_kind == 0 ? hd.g : S.g()[i];
-    }
-
-    // ---- pass A: values, gate, column sum S^T k
-    // packed: T holds the stored values V (codes or fp16) and mr the per-row
-    // multiplier M (a_i = r_i g_i, or g_i for a pivot row); the column sum
-    // is accumulated in fp64 from the exact per-row factors (see unpack_hi),
-    // in two halves of 8 columns to keep the accumulators few.
-    // fp32: T holds the gated state g_i S_ij and the column sum is fp32.
-    float2 T[G::RPT][8];
-    float mr[G::RPT];
-    float2 part[8];
-    float P;
-    if (PACKED) {
-      double kap[G::RPT];
-      double off = 0.0;
-      bool bad = false;
-#pragma unroll
-      for (int r = 0; r < G::RPT; ++r) {
-        const int i = r * G::NG + rg;
-        const uint8_t code = S.row_code()[i];
-        if (code == ROW_PIVOT) {
-          mr[r] = gr[r];
-          kap[r] = (double)gr[r] * (double)kr[r];
-        } else {
-          const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
-          mr[r] = __fmul_rn(R, gr[r]);
-          const int E = code == 8 ? 12 : code;  // FieldPos<code>::E
-          kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << E);
-          off = off + (1.0 + (double)(1 << (code - 1)) / (double)(1 << E)) * kap[r];
-        }
-        bad |= !isfinite(mr[r]) || !isfinite(kr[r]);
-      }
-      double* red64 = reinterpret_cast<double*>(red);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        double acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-#pragma unroll
-        for (int r = 0; r < G::RPT; ++r) {
-          const int i = r * G::NG + rg;
-          const uint8_t code = S.row_code()[i];
-          const uint8_t* row = S.rec() + S.row_off()[i];
-          // unpack through temporaries: writing T[r] from inside the width
-          // switch would push the whole tile into local memory
-          float2 vt[8];
-          uint32_t xh[16];
-          unpack_hi(row, code, cc, vt, xh);
-#pragma unroll
-          for (int p = 0; p < 4; ++p) T[r][4 * half + p] = vt[4 * half + p];
-          if (code == ROW_PIVOT) {
-#pragma unroll
-            for (int p = 0; p < 4; ++p) bad |= !isfinite(vt[4 * half + p].x) || !isfinite(vt[4 * half + p].y);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[8 * half + j], 0), kap[r], acc[j]);
-        }
-        deposit_f64<D>(red64, rg, cc, half, acc, off);
-      }
-      if (bad) nf_sh = 1;
-      P = column_total_f64<D>(red64);
-    } else {
-#pragma unroll
-      for (int r = 0; r < G::RPT; ++r) {
-        const int i = r * G::NG + rg;
-        const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          float4 x = src[p];
-          T[r][2 * p] = __fmul2_rn(make_float2(x.x, x.y), f2(gr[r]));
-          T[r][2 * p + 1] = __fmul2_rn(make_float2(x.z, x.w), f2(gr[r]));
-        }
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-          part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
-      }
-      P = column_sum<D>(red, rg, cc, part);
-    }
-    if ((tid & 1) == 0) {
-      const int j = tid >> 1;
-      float wj;
-      if (PACKED) {
-        const float p = __fmul_rn(S.c()[j], P);
-        const float u = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], p));
-        wj = __fmul_rn(u, S.ic()[j]);
-        if (!isfinite(wj)) nf_sh = 1;
-      } else {
-        wj = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
-      }
-      wsh[j] = wj;
-    }
-    __syncthreads();
-    const bool finite = nf_sh == 0;
-    float2 W[8];
-    {
-      const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float4 x = wsrc[p];
-        W[2 * p] = make_float2(x.x, x.y);
-        W[2 * p + 1] = make_float2(x.z, x.w);
-      }
-    }
-    // ---- pass B: gate + delta update (one rounding), partial S^T q
-#pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        if (PACKED) {
-          const float2 kw = __fmul2_rn(f2(kr[r]), W[p]);
-          T[r][p] = __ffma2_rn(T[r][p], f2(mr[r]), kw);
-        } else {
-          T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
-        }
-        part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr[r])) : __ffma2_rn(T[r][p], f2(qr[r]), part[p]);
-      }
-    }
-    {
-      const float O = column_sum<D>(red, rg, cc, part);
-      if ((tid & 1) == 0) {
-        const int j = tid >> 1;
-        const float oj = PACKED ? __fmul_rn(S.c()[j], O) : O;
-        if (oj != oj) st |= ST_NAN;
-        o[j] = oj;
-      }
-    }
-    // ---- requantize (or store fp32) into the stage record, in place
-    if (PACKED) {
-      st |= requant_rows<D>(S.rec(), S.row_off(), S.row_code(), S.phi(), rg, cc, finite, T);
-    } else {
-#pragma unroll
-      for (int r = 0; r < G::RPT; ++r) {
-        const int i = r * G::NG + rg;
-        float4* dst = reinterpret_cast<float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-          dst[p] = make_float4(T[r][2 * p].x, T[r][2 * p].y, T[r][2 * p + 1].x, T[r][2 * p + 1].y);
-      }
+    switch (PACKED ? hd.kind : 0) {
+      case 8: tile_body<D, PACKED, (PACKED ? 8 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      case 6: tile_body<D, PACKED, (PACKED ? 6 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      case 4: tile_body<D, PACKED, (PACKED ? 4 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      case 2: tile_body<D, PACKED, (PACKED ? 2 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      case ROW_PIVOT: tile_body<D, PACKED, (PACKED ? ROW_PIVOT : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      default: tile_body<D, PACKED, 0>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -931,7 +970,7 @@ __global__ void __launch_bounds__(Geo<D>::NT) k_quantize(const QuantArgs a) {
     }
   }
   __syncthreads();
-  uint32_t st = requant_rows<D>(rec, row_off, row_code, phi, rg, cc, false, T);
+  uint32_t st = requant_rows<D, 0>(rec, row_off, row_code, phi, rg, cc, false, T);
   __syncthreads();
   uint8_t* dst = a.pool + (uint64_t)slot * a.slot_bytes + a.t.rec_off[h];
   for (uint32_t x = tid * 16; x < rb; x += G::NT * 16) *reinterpret_cast<uint4*>(dst + x) = *reinterpret_cast<uint4*>(rec + x);
