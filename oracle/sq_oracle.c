@@ -52,7 +52,8 @@
  *   7. s_i   = fp32(fp32(phi_i m_i) / qmax_i); r'_i = fp16 of s_i rounded
  *      toward +inf (saturating at 65504); ir_i = 0 if r'_i == 0 else
  *      fp32(1 / r'_i)
- *   8. q'_ij = RNE(min(max(fp32(T'_ij * ir_i), -qmax), qmax))
+ *   8. q'_ij = min(max(RNE(T'_ij * ir_i), -qmax), qmax), the product taken
+ *      exactly (no fp32 rounding before the rounding to an integer)
  *   9. pivot rows: h'_ij = fp16 round-to-nearest-even of T'_ij, saturating
  *      at +-65504; a NaN stores 0.
  *  A row whose m_i is NaN stores r' = 0 and all codes 0 (status bit 0).
@@ -283,12 +284,14 @@ static uint32_t store_T(const sqo_desc *D, int h, uint8_t *rec, const float *T) 
     wr16(rec + 2 * i, rb);
     float r = sqo_f16_to_f32(rb);
     float ir = (r == 0.0f) ? 0.0f : 1.0f / r;
-    /* 9. codes: round half to even after clamping to the symmetric range */
+    /* 8. codes: the integer nearest to the exact product T' * ir (ties to
+     * even; the product of two floats is exact in double), clamped to the
+     * symmetric range */
     for (int j = 0; j < d; j++) {
-      float y = t[j] * ir;
-      if (y > (float)qm) y = (float)qm;
-      if (y < -(float)qm) y = -(float)qm;
-      sqo_put_code(row, b, j, (int)nearbyintf(y));
+      double y = nearbyint((double)t[j] * (double)ir);
+      if (y > (double)qm) y = (double)qm;
+      if (y < -(double)qm) y = -(double)qm;
+      sqo_put_code(row, b, j, (int)y);
     }
   }
   return st;

@@ -370,17 +370,22 @@ __device__ __forceinline__ void load_row(const uint8_t* row, uint8_t code, int c
 }
 
 // Requantize one row chunk of T' with inverse scale `ir` and write it back.
+// fma(T', ir, 2^23 + 2^(b-1)) rounds the exact product T' * ir to the
+// nearest integer (ties to even) in the window [2^23, 2^24) where floats
+// are integers; outside that window the value lies beyond the clamp bounds
+// whichever way it rounds, so clamping afterwards gives exactly the clamped
+// nearest integer. The result's low b bits are then the stored field.
 template <int B>
 __device__ __forceinline__ void store_row_q(uint8_t* row, int cc, float ir, const float2 (&t)[8]) {
   const float qm = (float)((1 << (B - 1)) - 1);
   const float magic = 8388608.0f + (float)(1 << (B - 1));
+  const float lo = magic - qm, hi = magic + qm;
   uint32_t fb[16];
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    float2 y = __fmul2_rn(t[p], f2(ir));
-    y.x = fminf(fmaxf(y.x, -qm), qm);
-    y.y = fminf(fmaxf(y.y, -qm), qm);
-    float2 n = __fadd2_rn(y, f2(magic));  // rounds to the nearest integer, ties to even
+    float2 n = __ffma2_rn(t[p], f2(ir), f2(magic));
+    n.x = fminf(fmaxf(n.x, lo), hi);
+    n.y = fminf(fmaxf(n.y, lo), hi);
     fb[2 * p] = __float_as_uint(n.x);
     fb[2 * p + 1] = __float_as_uint(n.y);
   }
@@ -883,7 +888,9 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
       case 6: tile_body<D, PACKED, (PACKED ? 6 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
       case 4: tile_body<D, PACKED, (PACKED ? 4 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
       case 2: tile_body<D, PACKED, (PACKED ? 2 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-      case ROW_PIVOT: tile_body<D, PACKED, (PACKED ? ROW_PIVOT : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
+      case ROW_PIVOT:
+        tile_body<D, PACKED, (PACKED ? ROW_PIVOT : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st);
+        break;
       default: tile_body<D, PACKED, 0>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
     }
     fence_proxy_async_smem();
@@ -892,7 +899,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
       nf_sh = 0;  // every read of this tile's flag happened before the barrier above
       bulk_s2g(hd.dst, S.rec(), hd.bytes);
       bulk_commit();
-      bulk_wait_read_all();
+      bulk_wait_read_all();  // the stage may be refilled once the store has read it
       if (tile + a.nstage < t1) {
         const TileScalars cur = pre;
         pre = load_scalars<D>(a, tile + a.nstage + 1, t1, PACKED);

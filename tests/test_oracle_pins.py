@@ -286,9 +286,9 @@ def test_quantizer_error_bound(oracle_mod, gate_kind):
 def test_requantization_bruteforce_tiny_tiles(oracle_mod):
     """2x2 and 4x4 tiles: every row scale is the smallest fp16 not below
     fp32(fp32(phi m)/qmax) (enumeration of all fp16 values), and every code
-    is the nearest integer (ties to even) to fp32(T * fp32(1/r)) within
-    [-qmax, qmax] (enumeration of all codes). The exact argmin of |T - r q|
-    agrees except within 2^-18 of a tie."""
+    is the integer in [-qmax, qmax] nearest (ties to even) to the exact
+    product T * fp32(1/r) (enumeration of all codes, exact rationals). The
+    exact argmin of |T - r q| agrees except within 2^-18 of a tie."""
     vals, _ = fp16_all_finite()
     rng = np.random.default_rng(60)
     near_ties = 0
@@ -317,8 +317,8 @@ def test_requantization_bruteforce_tiny_tiles(oracle_mod):
                         ir = np.float32(0) if r32 == 0 else np.float32(1) / r32
                         cand = np.arange(-qm, qm + 1)
                         for j in range(d):
-                            y = np.float64(T[i, j] * ir)
-                            dist = np.abs(cand - y)
+                            y = Fraction(float(T[i, j])) * Fraction(float(ir))
+                            dist = np.array([abs(y - c) for c in cand])
                             best = cand[dist == dist.min()]
                             best = best[best % 2 == 0] if len(best) > 1 else best
                             assert codes[i, j] == best[0]
@@ -473,3 +473,22 @@ def test_workload_recipes_match_configs():
         assert np.all((beta > 0) & (beta < 1))
         hl = cal.half_life
         assert hl.min() >= 1.0 and hl.max() <= cfg.half_life_max
+
+
+def test_code_rounds_the_exact_product(oracle_mod):
+    """r = 3 (row max 381 at 8 bits), so ir = fp32(1/3) = 0.3333333432...;
+    T = 151.5 gives the exact product 50.5000015..., whose nearest integer is
+    51, while rounding the product to fp32 first lands on the tie 50.5 and
+    then on the even 50. The code is 51."""
+    d = 4
+    o_ = oracle_mod.Oracle(1, 1, 1, d, 0, np.array([8], np.int8), np.array([0], np.uint8),
+                           np.ones((1, d), np.float32), np.ones((1, d), np.float32))
+    S = np.zeros((1, 1, d, d), np.float32)
+    S[0, 0, 0, 0] = 381.0
+    S[0, 0, 0, 1] = 151.5
+    pool = o_.new_pool()
+    o_.quantize(pool, S)
+    assert o_.row_scales(pool, 0, 0)[0].view(np.float16) == np.float16(3.0)
+    ir = np.float32(1) / np.float32(3)
+    assert np.float32(np.float32(151.5) * ir) == np.float32(50.5)
+    assert o_.codes(pool, 0, 0)[0, :2].tolist() == [127, 51]
