@@ -145,10 +145,21 @@ def run_ours(args, rank, world, local_rank):
     pool = sp.new_pool()
     sp.quantize_state(pool, S)
     torch.cuda.synchronize()
+    setup_status = sp.get_status()
     NI = 8
     host_inputs = [w.step_inputs(t) for t in range(NI)]
     dev_inputs = [[torch.from_numpy(x).to(dev) for x in xs] for xs in host_inputs]
     stream = torch.cuda.current_stream()
+    if args.profile:
+        # profiling mode: the same prepared state, N packed steps, no timing
+        for i in range(args.profile):
+            sp.decode_step(pool, *dev_inputs[i % NI], o)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_steps": args.profile, "status_after_setup": setup_status,
+                          "status_bits": sp.get_status()}), flush=True)
+        sp.close()
+        fp.close()
+        return
 
     def barrier():
         if dist is not None:
@@ -243,7 +254,8 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "k_decode_step<128,packed>", "algorithmic_bytes_per_launch": bytes_launch,
                      "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
-                  "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_bits": st_bits},
+                  "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
+                  "status_bits": st_bits},
         "fp32_state": {"value": world * units * max(4, args.steps // 4) / (fp_total / 1e3),
                        "kernel_ms": fp_kern, "achieved_gbs": fp_bytes / (fp_kern / 1e3) / 1e9,
                        "frac": fp_bytes / (fp_kern / 1e3) / 1e9 / peak,
@@ -317,6 +329,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-requests", type=int, default=48)
     ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--profile", type=int, default=0,
+                    help="prepare the workload, run this many packed steps untimed, exit (for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
