@@ -164,6 +164,37 @@ sq_status sq_get_status(sq_handle* h, void* stream, uint32_t* bits, int32_t clea
 /* Number of kernel launches this handle has issued (host-side counter). */
 uint64_t sq_launch_count(const sq_handle* h);
 
+/* Decode step that allocates nothing. The method's paper has no
+ * counterpart; this entry point exists for callers that cannot allocate
+ * device memory: a serving engine whose allocator has already reserved the
+ * GPU's memory for its own pools (a cudaMalloc behind its back would fail
+ * or fragment it), or a latency-critical caller that cannot afford the
+ * device synchronization cudaMalloc may imply. It does the same step as
+ * sq_decode_step on a packed pool laid out exactly as sq_state_alloc lays
+ * it out for the same `desc` and `calib`, but without a handle:
+ *   - the per-head tables (record and row offsets, widths, c, 1/c, phi)
+ *     are rebuilt on the host from `calib` at every call and copied into a
+ *     fixed 128 KiB array in device memory that this library declares at
+ *     file scope (every GPU that loads the library holds it until the
+ *     process exits); nothing is allocated on the device or the host heap;
+ *   - limits: packed pools only, h_v <= SQ_NOALLOC_MAX_HEADS, and the tables
+ *     must fit the array (h_v * d <= 8192 always does); larger shapes are
+ *     rejected with SQ_ERR_UNSUPPORTED and a message;
+ *   - the first call on a device looks up the array's device address and
+ *     sets the kernels' shared-memory limit for that device; make that
+ *     first call before any stream capture;
+ *   - every call shares the one array, which keeps the last call's tables:
+ *     calls on the same device serialize on the host, but calls whose GPU
+ *     work overlaps (different streams, or a later call before the earlier
+ *     one's kernel ran) race on the array;
+ *   - status: device pointer to a uint32 the kernel ORs SQ_STATUS_* bits
+ *     into (the caller clears it), or NULL to discard the bits.
+ * Other arguments as in sq_decode_step. */
+#define SQ_NOALLOC_MAX_HEADS 64
+sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_calib* calib, void* pool, const float* q,
+                                 const float* k, const float* v, const float* beta, const float* g, float* o,
+                                 const int32_t* slot_ids, int32_t B, uint32_t* status, void* stream);
+
 /* Message for the last non-OK return on this host thread ("" if none). */
 const char* sq_last_error(void);
 

@@ -30,6 +30,8 @@ SQ_STATUS_SATURATED = 2
 SQ_STATUS_BAD_SLOT = 4
 SQ_STATUS_TIMEOUT = 8
 
+SQ_NOALLOC_MAX_HEADS = 64
+
 
 class SQError(RuntimeError):
     def __init__(self, code: int, msg: str):
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
     L.sq_last_error.restype = ctypes.c_char_p
     L.sq_version.argtypes = []
     L.sq_version.restype = ctypes.c_char_p
+    L.sq_decode_step_noalloc.argtypes = [ctypes.POINTER(StateDesc), ctypes.POINTER(Calib)] + [P] * 8 + [I32, P, P]
+    L.sq_decode_step_noalloc.restype = ctypes.c_int
     for name in ("sq_state_alloc", "sq_state_free", "sq_quantize_state", "sq_decode_step",
                  "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status"):
         getattr(L, name).restype = ctypes.c_int
@@ -145,6 +149,13 @@ def sq_get_status(h, stream: int, clear: bool = True) -> int:
 
 def sq_launch_count(h) -> int:
     return int(lib().sq_launch_count(h))
+
+
+def sq_decode_step_noalloc(desc: StateDesc, calib: Calib, pool, q, k, v, beta, g, o, slot_ids, B, status,
+                           stream) -> None:
+    """The decode step without a handle and without any allocation (see include/sq.h)."""
+    check(lib().sq_decode_step_noalloc(ctypes.byref(desc), ctypes.byref(calib), pool, q, k, v, beta, g, o,
+                                       slot_ids, B, status, stream))
 
 
 def sq_version() -> str:

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <mutex>
 #include <vector>
 
 #include "sq.h"
@@ -474,3 +475,215 @@ sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, cons
 }
 
 }  // extern "C"
+
+// ===================================================================
+// Decode step that allocates nothing (sq_decode_step_noalloc).
+//
+// The regular path keeps its per-head tables (record offsets, row offsets,
+// widths, c, 1/c, phi, the status word) in device memory that
+// sq_state_alloc obtains with cudaMalloc. Here the same tables live in one
+// file-scope __device__ array, rebuilt on every call; nothing is allocated
+// on the device or the host heap.
+// ===================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 128 * 1024;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Host staging for the tables (the copy from pageable memory returns only
+// after the data has left this buffer, so it can be reused by the next call).
+static uint8_t g_noalloc_host[kNoAllocScratchBytes];
+static std::mutex g_noalloc_mutex;
+
+constexpr int kMaxDevices = 64;
+struct NoAllocDevice {
+  bool ready = false;
+  uint8_t* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int num_sms = 0, sm_smem = 0, optin_smem = 0;
+};
+static NoAllocDevice g_noalloc_dev[kMaxDevices];
+
+// Once per device, with that device current: the device address of the
+// scratch array (host code must not use the symbol itself) and the launch
+// limits. Runs inside the first call on the device.
+sq_status noalloc_setup(int dev, NoAllocDevice** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(SQ_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
+  NoAllocDevice& nd = g_noalloc_dev[dev];
+  if (!nd.ready) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    nd.scratch = static_cast<uint8_t*>(p);
+    e = cudaDeviceGetAttribute(&nd.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nd.sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nd.optin_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = allow_all<128>(nd.optin_smem);
+    if (e == cudaSuccess) e = allow_all<64>(nd.optin_smem);
+    if (e == cudaSuccess) e = allow_all<32>(nd.optin_smem);
+    if (e != cudaSuccess) return cuda_fail(e, "no-alloc set-up");
+    nd.ready = true;
+  }
+  *out = &nd;
+  return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_calib* calib, void* pool,
+                                             const float* q, const float* k, const float* v, const float* beta,
+                                             const float* g, float* o, const int32_t* slot_ids, int32_t B,
+                                             uint32_t* status, void* stream) {
+  g_last_error.clear();
+  sq_status s = validate_desc(desc);
+  if (s != SQ_OK) return s;
+  if (desc->fmt != SQ_FMT_PACKED) return fail(SQ_ERR_UNSUPPORTED, "the no-alloc step takes packed pools only");
+  const int d = desc->d_k, hv = desc->h_v;
+  if (hv > SQ_NOALLOC_MAX_HEADS)
+    return fail(SQ_ERR_UNSUPPORTED, "no-alloc step: h_v = %d exceeds its maximum of %d heads", hv,
+                SQ_NOALLOC_MAX_HEADS);
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  const bool per_row = desc->gate == SQ_GATE_KEY_CHANNEL;
+  const size_t n_units = per_row ? (size_t)hv * d : (size_t)hv;
+  if (!calib || !calib->unit_bits || !calib->pivot_mask || !calib->col_scale || !calib->row_impact)
+    return fail(SQ_ERR_INVALID_ARG, "packed format needs all four calibration arrays");
+  for (size_t u = 0; u < n_units; ++u) {
+    const int b = calib->unit_bits[u];
+    if (!calib->pivot_mask[u] && b != 2 && b != 4 && b != 6 && b != 8)
+      return fail(SQ_ERR_INVALID_ARG, "unit %zu: bit width %d not in {2,4,6,8}", u, b);
+  }
+  const size_t nhd = (size_t)hv * d;
+  for (size_t x = 0; x < nhd; ++x) {
+    const float c = calib->col_scale[x], p = calib->row_impact[x];
+    if (!std::isfinite(c) || !(c > 0.0f) || !std::isfinite(1.0f / c))
+      return fail(SQ_ERR_INVALID_ARG, "col_scale[%zu] = %g is not finite > 0", x, c);
+    if (!std::isfinite(p) || !(p > 0.0f)) return fail(SQ_ERR_INVALID_ARG, "row_impact[%zu] = %g is not finite > 0", x, p);
+  }
+  if (B == 0) return SQ_OK;
+  if ((int64_t)B * hv > (int64_t)INT32_MAX / 2) return fail(SQ_ERR_INVALID_ARG, "B too large");
+  SQ_CHECK_PTR(pool, "pool");
+  SQ_CHECK_PTR(q, "q");
+  SQ_CHECK_PTR(k, "k");
+  SQ_CHECK_PTR(v, "v");
+  SQ_CHECK_PTR(o, "o");
+  if (!beta || !g) return fail(SQ_ERR_INVALID_ARG, "beta/g is NULL");
+  if (per_row && !aligned16(g)) return fail(SQ_ERR_INVALID_ARG, "g is not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(SQ_ERR_INVALID_ARG, "beta/g not 4-byte aligned");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  if (status && (reinterpret_cast<uintptr_t>(status) & 3u)) return fail(SQ_ERR_INVALID_ARG, "status misaligned");
+
+  // table layout inside the scratch array (same tables as a handle's)
+  const size_t o_rec_off = 0;
+  const size_t o_rec_bytes = round_up(o_rec_off + 4 * (size_t)hv, 16);
+  const size_t o_col = round_up(o_rec_bytes + 4 * (size_t)hv, 16);
+  const size_t o_icol = round_up(o_col + 4 * nhd, 16);
+  const size_t o_phi = round_up(o_icol + 4 * nhd, 16);
+  const size_t o_row_off = round_up(o_phi + 4 * nhd, 16);
+  const size_t o_row_code = round_up(o_row_off + 2 * nhd, 16);
+  const size_t o_head_kind = round_up(o_row_code + nhd, 16);
+  const size_t o_status = round_up(o_head_kind + (size_t)hv, 16);
+  const size_t total = round_up(o_status + 16, 16);
+  if (total > kNoAllocScratchBytes)
+    return fail(SQ_ERR_UNSUPPORTED, "no-alloc step: tables need %zu bytes, above its %zu-byte scratch", total,
+                kNoAllocScratchBytes);
+
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "no usable CUDA device");
+  NoAllocDevice* nd = nullptr;
+  s = noalloc_setup(dev, &nd);
+  if (s != SQ_OK) return s;
+
+  uint8_t* host = g_noalloc_host;
+  memset(host, 0, total);
+  uint32_t* rec_off = reinterpret_cast<uint32_t*>(host + o_rec_off);
+  uint32_t* rec_bytes = reinterpret_cast<uint32_t*>(host + o_rec_bytes);
+  float* col = reinterpret_cast<float*>(host + o_col);
+  float* icol = reinterpret_cast<float*>(host + o_icol);
+  float* phi = reinterpret_cast<float*>(host + o_phi);
+  uint16_t* row_off = reinterpret_cast<uint16_t*>(host + o_row_off);
+  uint8_t* row_code = host + o_row_code;
+  uint8_t* head_kind = host + o_head_kind;
+  uint64_t off = 0, max_rec = 0;
+  for (int hh = 0; hh < hv; ++hh) {
+    uint64_t n = 2ull * d;
+    for (int i = 0; i < d; ++i) {
+      const size_t u = per_row ? (size_t)hh * d + i : (size_t)hh;
+      const bool piv = calib->pivot_mask[u] != 0;
+      const uint8_t code = piv ? sqk::ROW_PIVOT : (uint8_t)calib->unit_bits[u];
+      row_off[(size_t)hh * d + i] = (uint16_t)n;
+      row_code[(size_t)hh * d + i] = code;
+      n += piv ? 2ull * d : (uint64_t)d * code / 8;
+    }
+    n = round_up(n, 16);
+    rec_off[hh] = (uint32_t)off;
+    rec_bytes[hh] = (uint32_t)n;
+    if (n > max_rec) max_rec = n;
+    off += n;
+    uint8_t kind = row_code[(size_t)hh * d];
+    for (int i = 1; i < d && kind; ++i)
+      if (row_code[(size_t)hh * d + i] != kind) kind = 0;
+    head_kind[hh] = kind;
+  }
+  for (size_t x = 0; x < nhd; ++x) {
+    col[x] = calib->col_scale[x];
+    volatile float c = col[x];
+    icol[x] = 1.0f / c;  // IEEE single-precision division
+    phi[x] = calib->row_impact[x];
+  }
+  cudaStream_t st = as_stream(stream);
+  e = cudaMemcpyAsync(nd->scratch, host, total, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "uploading no-alloc tables");
+
+  sqk::StepArgs a{};
+  a.pool = static_cast<uint8_t*>(pool);
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
+  a.slots = slot_ids;
+  a.B = B; a.h_v = hv; a.h_k = desc->h_k; a.n_slots = desc->n_slots; a.gate_kind = desc->gate;
+  a.slot_bytes = off;
+  a.t.rec_off = reinterpret_cast<const uint32_t*>(nd->scratch + o_rec_off);
+  a.t.rec_bytes = reinterpret_cast<const uint32_t*>(nd->scratch + o_rec_bytes);
+  a.t.col = reinterpret_cast<const float*>(nd->scratch + o_col);
+  a.t.icol = reinterpret_cast<const float*>(nd->scratch + o_icol);
+  a.t.phi = reinterpret_cast<const float*>(nd->scratch + o_phi);
+  a.t.row_off = reinterpret_cast<const uint16_t*>(nd->scratch + o_row_off);
+  a.t.row_code = reinterpret_cast<const uint8_t*>(nd->scratch + o_row_code);
+  a.t.head_kind = reinterpret_cast<const uint8_t*>(nd->scratch + o_head_kind);
+  a.t.status = status ? status : reinterpret_cast<uint32_t*>(nd->scratch + o_status);
+
+  // launch plan (same rule as a handle's)
+  a.rec_cap = (uint32_t)round_up(max_rec, 128);
+  a.stage_bytes = (uint32_t)round_up(a.rec_cap + 31u * d + 32u, 128);
+  const size_t red = (size_t)32 * d * 8;
+  const size_t budget = (size_t)nd->sm_smem / 2 - 2048 - 1024;
+  int ns = (int)((budget - red) / a.stage_bytes);
+  if (ns > 4) ns = 4;
+  if (ns < 1) ns = 1;
+  size_t smem = (size_t)ns * a.stage_bytes + red;
+  const size_t dyn_max = (size_t)nd->optin_smem - 1024;
+  while (smem > dyn_max && ns > 1) {
+    --ns;
+    smem = (size_t)ns * a.stage_bytes + red;
+  }
+  if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
+  a.nstage = ns;
+  int blocks = 0;
+  if (d == 128) e = occupancy<128, true>(&blocks, smem);
+  else if (d == 64) e = occupancy<64, true>(&blocks, smem);
+  else e = occupancy<32, true>(&blocks, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+  if (blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+  const int n_tiles = B * hv;
+  const int grid = n_tiles < blocks * nd->num_sms ? n_tiles : blocks * nd->num_sms;
+  if (!status) {
+    e = cudaMemsetAsync(nd->scratch + o_status, 0, 4, st);  // the scratch status word starts at zero
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch status word");
+  }
+  if (d == 128) sqk::k_decode_step<128, true><<<grid, threads_of(128), smem, st>>>(a);
+  else if (d == 64) sqk::k_decode_step<64, true><<<grid, threads_of(64), smem, st>>>(a);
+  else sqk::k_decode_step<32, true><<<grid, threads_of(32), smem, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching the no-alloc decode step");
+  return SQ_OK;
+}
