@@ -56,6 +56,7 @@ struct sq_handle {
   int step_grid = 0;
   int nstage = 0;
   uint32_t rec_cap = 0, stage_bytes = 0;
+  uint64_t stage_rec = 0;  // largest record that goes through a stage
   size_t step_smem = 0;
   uint64_t launches = 0;
 };
@@ -87,61 +88,111 @@ cudaError_t allow_max_smem(K kernel, int max_smem) {
 
 template <int D>
 cudaError_t allow_all(int max_smem) {
-  cudaError_t e = allow_max_smem(sqk::k_decode_step<D, true>, max_smem);
-  if (e == cudaSuccess) e = allow_max_smem(sqk::k_decode_step<D, false>, max_smem);
+  cudaError_t e = allow_max_smem(sqk::k_decode_step_packed<D>, max_smem);
+  if (e == cudaSuccess) e = allow_max_smem(sqk::k_decode_step_fp32<D>, max_smem);
   if (e == cudaSuccess) e = allow_max_smem(sqk::k_quantize<D>, max_smem);
   if (e == cudaSuccess) e = allow_max_smem(sqk::k_dequantize<D>, max_smem);
   return e;
 }
 
-template <int D, bool PACKED>
-cudaError_t occupancy(int* blocks, size_t smem) {
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, sqk::k_decode_step<D, PACKED>, sqk::Geo<D>::NT,
-                                                       smem);
+template <int D>
+const void* step_kernel(bool packed) {
+  return packed ? reinterpret_cast<const void*>(sqk::k_decode_step_packed<D>)
+                : reinterpret_cast<const void*>(sqk::k_decode_step_fp32<D>);
 }
 
-// Choose stages and grid for the persistent step kernel.
+const void* step_kernel_of(int d, bool packed) {
+  switch (d) {
+    case 128: return step_kernel<128>(packed);
+    case 64: return step_kernel<64>(packed);
+    default: return step_kernel<32>(packed);
+  }
+}
+
+// Launch plan of the persistent step kernel.
+struct StepPlan {
+  uint32_t rec_cap = 0, stage_bytes = 0;
+  int nstage = 0;
+  size_t smem = 0;
+  int blocks = 0;  // CTAs per SM
+};
+
+// Packed pools: a stage holds one record (every head except the all-pivot
+// ones, which the kernel reads in place) plus the tile's vectors; the S^T k
+// and o partials share one buffer of 32 d fp64 values. The pipeline needs
+// at least 2 stages. Preference: as many CTAs per SM as registers allow (at
+// most 3, with 2 stages), then as many stages as fit (at most 4). FP32
+// pools: 1 CTA per SM, up to 4 stages.
+sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int optin_smem, int reserved_smem,
+                      StepPlan* p) {
+  const void* kern = step_kernel_of(d, packed);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+  const size_t static_smem = fa.sharedSizeBytes;
+  p->rec_cap = (uint32_t)round_up(stage_rec < 16 ? 16 : stage_rec, 128);
+  p->stage_bytes = (uint32_t)round_up(p->rec_cap + 31u * d + 32u, 128);  // + vectors, tables, header
+  const int NG = 32;  // row groups per CTA: 32 for every supported d
+  const size_t red = (size_t)NG * d * (packed ? 8 : 4);
+  const size_t dyn_max = (size_t)optin_smem - static_smem;
+  const int min_ns = packed ? 2 : 1;
+  // CTAs per SM allowed by registers and threads alone
+  int by_regs = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&by_regs, kern, threads_of(d), 0);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+  int first = packed ? 3 : 1;
+  if (by_regs >= 1 && by_regs < first) first = by_regs;
+  p->nstage = 0;
+  for (int want = first; want >= 1 && p->nstage == 0; --want) {
+    const long budget = (long)sm_smem / want - reserved_smem - (long)static_smem;
+    if (budget < (long)red) continue;
+    int ns = (int)((size_t)(budget - (long)red) / p->stage_bytes);
+    if (ns > 4) ns = 4;
+    if (want == 3 && ns > 2) ns = 2;
+    if (ns < min_ns) continue;
+    const size_t smem = (size_t)ns * p->stage_bytes + red;
+    if (smem > dyn_max) continue;
+    p->nstage = ns;
+    p->smem = smem;
+  }
+  if (p->nstage == 0) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p->blocks, kern, threads_of(d), p->smem);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+  if (p->blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+  return SQ_OK;
+}
+
+// Largest record that goes through a stage: that of every head except the
+// all-pivot ones.
+uint64_t staged_record_bytes(const uint32_t* rec_bytes, const uint8_t* head_kind, int hv) {
+  uint64_t m = 0;
+  for (int hh = 0; hh < hv; ++hh)
+    if (head_kind[hh] != sqk::ROW_PIVOT && rec_bytes[hh] > m) m = rec_bytes[hh];
+  return m;
+}
+
+// Choose stages and grid for the persistent step kernel of a handle.
 sq_status plan_step(sq_handle* h) {
   const int d = h->d;
   const bool packed = h->desc.fmt == SQ_FMT_PACKED;
-  const uint32_t rec = packed ? (uint32_t)h->max_rec : (uint32_t)(4u * d * d);
-  h->rec_cap = (uint32_t)round_up(rec, 128);
-  h->stage_bytes = (uint32_t)round_up(h->rec_cap + 31u * d + 32u, 128);  // + per-tile header
-  const int NG = 32;  // row groups per CTA: 32 for every supported d
-  const size_t red = (size_t)NG * d * (packed ? 8 : 4);  // fp64 column partials when packed
-  int dev_max_smem = 0;
-  cudaError_t e = cudaDeviceGetAttribute(&dev_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  int optin = 0, sm_smem = 0, reserved = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, h->device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  int sm_smem = 0;
-  e = cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, h->device);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-  // target: 2 CTAs per SM for the packed kernel, 1 for fp32; 2..4 stages
-  const int want_ctas = packed ? 2 : 1;
-  const size_t static_smem = 2048;  // barriers, w vector, flags (upper bound)
-  const size_t budget = (size_t)sm_smem / want_ctas - static_smem - 1024 /* per-CTA reserve */;
-  int ns = (int)((budget - red) / h->stage_bytes);
-  if (ns > 4) ns = 4;
-  if (ns < 1) ns = 1;
-  size_t smem = (size_t)ns * h->stage_bytes + red;
-  const size_t dyn_max = (size_t)dev_max_smem - 1024;  // room for the static shared variables
-  while (smem > dyn_max && ns > 1) {
-    --ns;
-    smem = (size_t)ns * h->stage_bytes + red;
-  }
-  if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
-  h->nstage = ns;
-  h->step_smem = smem;
-  int blocks = 0;
-  if (d == 128) e = allow_all<128>(dev_max_smem);
-  else if (d == 64) e = allow_all<64>(dev_max_smem);
-  else e = allow_all<32>(dev_max_smem);
+  if (d == 128) e = allow_all<128>(optin);
+  else if (d == 64) e = allow_all<64>(optin);
+  else e = allow_all<32>(optin);
   if (e != cudaSuccess) return cuda_fail(e, "kernel attributes");
-  if (d == 128) e = packed ? occupancy<128, true>(&blocks, smem) : occupancy<128, false>(&blocks, smem);
-  else if (d == 64) e = packed ? occupancy<64, true>(&blocks, smem) : occupancy<64, false>(&blocks, smem);
-  else e = packed ? occupancy<32, true>(&blocks, smem) : occupancy<32, false>(&blocks, smem);
-  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
-  if (blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
-  h->step_grid = blocks * h->num_sms;
+  StepPlan p;
+  const uint64_t stage_rec = packed ? h->stage_rec : 4ull * d * d;
+  sq_status s = plan_kernel(d, packed, stage_rec, sm_smem, optin, reserved, &p);
+  if (s != SQ_OK) return s;
+  h->rec_cap = p.rec_cap;
+  h->stage_bytes = p.stage_bytes;
+  h->nstage = p.nstage;
+  h->step_smem = p.smem;
+  h->step_grid = p.blocks * h->num_sms;
   return SQ_OK;
 }
 
@@ -270,6 +321,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
       if (h->row_code[(size_t)hh * d + i] != k) k = 0;
     host[o_head_kind + hh] = k;
   }
+  h->stage_rec = packed ? staged_record_bytes(h->rec_bytes.data(), host.data() + o_head_kind, hv) : 0;
   e = cudaMalloc(&h->dev_block, total);
   if (e != cudaSuccess) {
     delete h;
@@ -389,13 +441,13 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
   cudaStream_t st = as_stream(stream);
   const bool packed = h->desc.fmt == SQ_FMT_PACKED;
   if (packed) {
-    if (h->d == 128) sqk::k_decode_step<128, true><<<grid, nt, h->step_smem, st>>>(a);
-    else if (h->d == 64) sqk::k_decode_step<64, true><<<grid, nt, h->step_smem, st>>>(a);
-    else sqk::k_decode_step<32, true><<<grid, nt, h->step_smem, st>>>(a);
+    if (h->d == 128) sqk::k_decode_step_packed<128><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step_packed<64><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step_packed<32><<<grid, nt, h->step_smem, st>>>(a);
   } else {
-    if (h->d == 128) sqk::k_decode_step<128, false><<<grid, nt, h->step_smem, st>>>(a);
-    else if (h->d == 64) sqk::k_decode_step<64, false><<<grid, nt, h->step_smem, st>>>(a);
-    else sqk::k_decode_step<32, false><<<grid, nt, h->step_smem, st>>>(a);
+    if (h->d == 128) sqk::k_decode_step_fp32<128><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step_fp32<64><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step_fp32<32><<<grid, nt, h->step_smem, st>>>(a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching the decode step");
@@ -499,7 +551,7 @@ constexpr int kMaxDevices = 64;
 struct NoAllocDevice {
   bool ready = false;
   uint8_t* scratch = nullptr;  // device address of g_noalloc_scratch on this device
-  int num_sms = 0, sm_smem = 0, optin_smem = 0;
+  int num_sms = 0, sm_smem = 0, optin_smem = 0, reserved_smem = 0;
 };
 static NoAllocDevice g_noalloc_dev[kMaxDevices];
 
@@ -517,6 +569,7 @@ sq_status noalloc_setup(int dev, NoAllocDevice** out) {
     e = cudaDeviceGetAttribute(&nd.num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nd.sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nd.optin_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nd.reserved_smem, cudaDevAttrReservedSharedMemoryPerBlock, dev);
     if (e == cudaSuccess) e = allow_all<128>(nd.optin_smem);
     if (e == cudaSuccess) e = allow_all<64>(nd.optin_smem);
     if (e == cudaSuccess) e = allow_all<32>(nd.optin_smem);
@@ -653,36 +706,24 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.t.status = status ? status : reinterpret_cast<uint32_t*>(nd->scratch + o_status);
 
   // launch plan (same rule as a handle's)
-  a.rec_cap = (uint32_t)round_up(max_rec, 128);
-  a.stage_bytes = (uint32_t)round_up(a.rec_cap + 31u * d + 32u, 128);
-  const size_t red = (size_t)32 * d * 8;
-  const size_t budget = (size_t)nd->sm_smem / 2 - 2048 - 1024;
-  int ns = (int)((budget - red) / a.stage_bytes);
-  if (ns > 4) ns = 4;
-  if (ns < 1) ns = 1;
-  size_t smem = (size_t)ns * a.stage_bytes + red;
-  const size_t dyn_max = (size_t)nd->optin_smem - 1024;
-  while (smem > dyn_max && ns > 1) {
-    --ns;
-    smem = (size_t)ns * a.stage_bytes + red;
-  }
-  if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
-  a.nstage = ns;
-  int blocks = 0;
-  if (d == 128) e = occupancy<128, true>(&blocks, smem);
-  else if (d == 64) e = occupancy<64, true>(&blocks, smem);
-  else e = occupancy<32, true>(&blocks, smem);
-  if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
-  if (blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
+  StepPlan p;
+  s = plan_kernel(d, true, staged_record_bytes(rec_bytes, head_kind, hv), nd->sm_smem, nd->optin_smem,
+                  nd->reserved_smem, &p);
+  if (s != SQ_OK) return s;
+  a.rec_cap = p.rec_cap;
+  a.stage_bytes = p.stage_bytes;
+  a.nstage = p.nstage;
+  const size_t smem = p.smem;
+  const int blocks = p.blocks;
   const int n_tiles = B * hv;
   const int grid = n_tiles < blocks * nd->num_sms ? n_tiles : blocks * nd->num_sms;
   if (!status) {
     e = cudaMemsetAsync(nd->scratch + o_status, 0, 4, st);  // the scratch status word starts at zero
     if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch status word");
   }
-  if (d == 128) sqk::k_decode_step<128, true><<<grid, threads_of(128), smem, st>>>(a);
-  else if (d == 64) sqk::k_decode_step<64, true><<<grid, threads_of(64), smem, st>>>(a);
-  else sqk::k_decode_step<32, true><<<grid, threads_of(32), smem, st>>>(a);
+  if (d == 128) sqk::k_decode_step_packed<128><<<grid, threads_of(128), smem, st>>>(a);
+  else if (d == 64) sqk::k_decode_step_packed<64><<<grid, threads_of(64), smem, st>>>(a);
+  else sqk::k_decode_step_packed<32><<<grid, threads_of(32), smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching the no-alloc decode step");
   return SQ_OK;

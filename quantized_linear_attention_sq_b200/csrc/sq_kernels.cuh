@@ -206,23 +206,33 @@ __device__ __forceinline__ void unpack16(const uint32_t* w, float2 (&f)[8]) {
   }
 }
 
-// Exponent E of the fp64 view of a field: the field sits at bits
-// [20-E, 20-E+B) of the word 0x3FF00000, so that, read as the high word of a
-// double (low word 0), the word is 1 + field * 2^-E exactly and, read as a
-// float, 1.875 + field * 2^-(E+3). 8-bit fields go to a byte boundary
-// (E = 12) so one byte permute places them; the others use E = B.
+// fp64 view of a b-bit field f for the S^T k column sum: the field is placed
+// at bits [20-E, 20-E+b) of a high word whose exponent field is 1023 + E, so
+// that this word over a zero low word is the double 2^E + f exactly. 8-bit
+// fields go to a byte boundary (E = 12), where one byte permute places them;
+// the other widths use E = b.
+//
+// Read as a float, the same word is v = 2^EF (1 + M0 2^-23) + f 2^(POS+EF-23)
+// (EF, M0: exponent and mantissa of the float view of EXP), so the code
+// q = f - 2^(b-1) is exactly fma(v, K, -C) with K = 2^(23-POS-EF) and
+// C = 2^(23-POS) + (M0 >> POS) + 2^(b-1), where M0 >> POS = ((1023+E) & 7) 2^E.
 template <int B>
 struct FieldPos {
   static constexpr int E = B == 8 ? 12 : B;
   static constexpr int POS = 20 - E;
+  static constexpr uint32_t EXP = (0x3FFu + (uint32_t)E) << 20;
+  static constexpr int EF = (int)((EXP >> 23) & 0xFFu) - 127;
+  static constexpr float K = (float)(1u << (23 - POS - EF));
+  static constexpr float C = (float)((1u << (23 - POS)) + ((0x3FFu + (uint32_t)E) & 7u) * (1u << E) + (1u << (B - 1)));
 };
 
 // Field j of a 16-code chunk held in b/2 words, in place as described above.
 template <int B>
 __device__ __forceinline__ uint32_t field_hi(const uint32_t* w, int j) {
   constexpr int POS = FieldPos<B>::POS;
+  constexpr uint32_t EXP = FieldPos<B>::EXP;
   if constexpr (B == 8) {
-    return __byte_perm(w[j >> 2], 0x3FF00000u, 0x7604u | ((uint32_t)(j & 3) << 4));
+    return __byte_perm(w[j >> 2], EXP, 0x7604u | ((uint32_t)(j & 3) << 4));
   } else {
     constexpr uint32_t MASK = ((1u << B) - 1u) << POS;
     const int bit = B * j;
@@ -233,55 +243,76 @@ __device__ __forceinline__ uint32_t field_hi(const uint32_t* w, int j) {
       x = sh >= POS ? (w[wi] >> (sh - POS)) : (w[wi] << (POS - sh));
     else
       x = __funnelshift_r(w[wi], w[wi + 1], sh - POS);  // a straddling field always has sh > POS
-    return 0x3FF00000u | (x & MASK);
+    return EXP | (x & MASK);
   }
 }
 
-// Pass-A unpack of one quantized 16-code chunk: the codes q as floats (exact)
-// and the high words of the doubles 1 + field * 2^-E that feed the fp64
-// column sum (with the per-row factor 2^E a k, minus (1 + 2^(B-1-E)) 2^E a k
-// per row, they give q a k up to fp64 rounding).
-template <int B>
-__device__ __forceinline__ void unpack_q_hi(const uint8_t* row, int cc, float2 (&V)[8], uint32_t (&xh)[16]) {
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(row + 2 * B * cc);
-  uint32_t w[B / 2];
+// Per-row constant of the fp64 column sum: a row of width b adds
+// (2^E + f) kap to every column, so (2^E + 2^(b-1)) kap is taken off once
+// per row to leave q kap (f = q + 2^(b-1)).
+__device__ __forceinline__ double code_offset(int code) {
+  const int E = code == 8 ? 12 : code;
+  return (double)((1 << E) + (1 << (code - 1)));
+}
+
+// The b/2 code words (quantized row, b in {2,4,6,8}) or 8 fp16-pair words
+// (pivot row) of the 16-column chunk cc of one row, from shared memory or,
+// for GLOBAL, from the pool itself. VEC: the chunk is aligned to its size
+// (up to 16 bytes), true for every row of a head of uniform width; rows of
+// mixed-width heads are only 4-byte aligned (d = 32: a 6-bit row is 24 B).
+template <int B, bool GLOBAL, bool VEC = true>
+__device__ __forceinline__ void chunk_words(const uint8_t* row, int cc, uint32_t (&w)[B / 2]) {
+  const uint8_t* p = row + 2 * B * cc;
+  if constexpr (!VEC) {
 #pragma unroll
-  for (int i = 0; i < B / 2; ++i) w[i] = src[i];
-  constexpr int E = FieldPos<B>::E;
-  const float S = (float)(1 << (E + 3));
-  const float C = 1.875f * S + (float)(1 << (B - 1));
+    for (int i = 0; i < B / 2; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  } else if constexpr (GLOBAL) {
+    static_assert(B % 8 == 0, "global rows are read in 16-byte pieces");
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const uint32_t h0 = field_hi<B>(w, 2 * p), h1 = field_hi<B>(w, 2 * p + 1);
-    xh[2 * p] = h0;
-    xh[2 * p + 1] = h1;
-    V[p] = __ffma2_rn(make_float2(__uint_as_float(h0), __uint_as_float(h1)), make_float2(S, S),
+    for (int q = 0; q < B / 8; ++q) {
+      uint4 x;
+      asm("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                   : "l"(p + 16 * q));
+      w[4 * q] = x.x; w[4 * q + 1] = x.y; w[4 * q + 2] = x.z; w[4 * q + 3] = x.w;
+    }
+  } else if constexpr (B == 8 || B == 16) {
+#pragma unroll
+    for (int q = 0; q < B / 8; ++q) {
+      const uint4 x = reinterpret_cast<const uint4*>(p)[q];
+      w[4 * q] = x.x; w[4 * q + 1] = x.y; w[4 * q + 2] = x.z; w[4 * q + 3] = x.w;
+    }
+  } else if constexpr (B == 4) {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x; w[1] = x.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < B / 2; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+  }
+}
+
+// High words of the fp64 views of the 8 values of half H of a chunk, and
+// the same 8 values as floats (codes q, or fp16 pivot values).
+template <int B, int H>
+__device__ __forceinline__ void hi_half_q(const uint32_t (&w)[B / 2], uint32_t (&xh)[8], float2 (&V)[4]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) xh[j] = field_hi<B>(w, 8 * H + j);
+  constexpr float K = FieldPos<B>::K, C = FieldPos<B>::C;
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    V[p] = __ffma2_rn(make_float2(__uint_as_float(xh[2 * p]), __uint_as_float(xh[2 * p + 1])), make_float2(K, K),
                       make_float2(-C, -C));
-  }
 }
-
-// Pass-A unpack of one fp16 pivot chunk: the values as floats and the high
-// words of the same values as doubles (an fp16 value has a zero low word).
-__device__ __forceinline__ void unpack_pivot_hi(const uint8_t* row, int cc, float2 (&V)[8], uint32_t (&xh)[16]) {
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(row + 32 * cc);
+// Pivot chunk: the fp16 values themselves (an fp16 value as a double has a
+// zero low word).
+template <int H>
+__device__ __forceinline__ void hi_half_pivot(const uint32_t (&w)[8], uint32_t (&xh)[8], float2 (&V)[4]) {
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    __half2 h2 = *reinterpret_cast<const __half2*>(src + p);
-    float2 x = __half22float2(h2);
+  for (int p = 0; p < 4; ++p) {
+    const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[4 * H + p]));
     V[p] = x;
     xh[2 * p] = (uint32_t)__double2hiint((double)x.x);
     xh[2 * p + 1] = (uint32_t)__double2hiint((double)x.y);
-  }
-}
-
-__device__ __forceinline__ void unpack_hi(const uint8_t* row, uint8_t code, int cc, float2 (&V)[8],
-                                          uint32_t (&xh)[16]) {
-  switch (code) {
-    case 8: unpack_q_hi<8>(row, cc, V, xh); break;
-    case 6: unpack_q_hi<6>(row, cc, V, xh); break;
-    case 4: unpack_q_hi<4>(row, cc, V, xh); break;
-    case 2: unpack_q_hi<2>(row, cc, V, xh); break;
-    default: unpack_pivot_hi(row, cc, V, xh); break;
   }
 }
 
@@ -410,10 +441,12 @@ __device__ __forceinline__ void store_row_zero(uint8_t* row, int B, int cc) {
   }
 }
 
-// fp16 pivot row: RNE with saturation at +-65504; NaN stores 0.
+// fp16 pivot row: RNE with saturation at +-65504; NaN stores 0. GLOBAL: the
+// row is in the pool (16-byte aligned chunks), else in shared memory.
+template <bool GLOBAL>
 __device__ __forceinline__ uint32_t store_row_pivot(uint8_t* row, int cc, const float2 (&t)[8]) {
   uint32_t st = 0;
-  uint32_t* dst = reinterpret_cast<uint32_t*>(row + 32 * cc);
+  uint32_t w[8];
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     float x0 = t[p].x, x1 = t[p].y;
@@ -422,7 +455,18 @@ __device__ __forceinline__ uint32_t store_row_pivot(uint8_t* row, int cc, const 
     if (fabsf(x0) > 65504.0f) { x0 = copysignf(65504.0f, x0); st |= ST_SAT; }
     if (fabsf(x1) > 65504.0f) { x1 = copysignf(65504.0f, x1); st |= ST_SAT; }
     __half2 h = __floats2half2_rn(x0, x1);
-    dst[p] = *reinterpret_cast<uint32_t*>(&h);
+    w[p] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  uint8_t* dst = row + 32 * cc;
+  if constexpr (GLOBAL) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16 * q), "r"(w[4 * q]),
+                   "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) reinterpret_cast<uint32_t*>(dst)[p] = w[p];
   }
   return st;
 }
@@ -507,7 +551,7 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
     const int code = KC ? KC : row_code[i];
     uint8_t* row = rec + row_offset<D, KC>(row_off, i);
     if (code == ROW_PIVOT) {
-      st |= store_row_pivot(row, cc, T[r]);
+      st |= store_row_pivot<false>(row, cc, T[r]);
     } else if (m[r] != m[r]) {  // a NaN in the row: scale 0, all codes 0
       store_row_zero(row, code, cc);
     } else {
@@ -526,19 +570,20 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
 // a thread's chunks are stored rotated by its column block (XOR swizzle) so
 // the eight lanes of a row write eight different bank groups. Then two
 // adjacent threads own one column (thread 2j and 2j+1 each add half of the
-// row groups) and combine with one shuffle. Returns the column total in
-// every thread of the pair; column = threadIdx.x >> 1. The caller syncs
-// before reusing `red`.
+// row groups) and combine with one shuffle; column = threadIdx.x >> 1.
 template <int D>
-__device__ __forceinline__ float column_sum(float* red, int rg, int cc, const float2 (&part)[8]) {
-  using G = Geo<D>;
-  static_assert(G::NT == 2 * D, "two threads per column");
+__device__ __forceinline__ void column_deposit(float* red, int rg, int cc, const float2 (&part)[8]) {
   const int sw = (cc >> 1) & 3;
 #pragma unroll
   for (int p = 0; p < 4; ++p)
     *reinterpret_cast<float4*>(red + rg * D + 16 * cc + 4 * (p ^ sw)) =
         make_float4(part[2 * p].x, part[2 * p].y, part[2 * p + 1].x, part[2 * p + 1].y);
-  __syncthreads();
+}
+
+template <int D>
+__device__ __forceinline__ float column_total(const float* red) {
+  using G = Geo<D>;
+  static_assert(G::NT == 2 * D, "two threads per column");
   const int j = threadIdx.x >> 1;
   const int hh = threadIdx.x & 1;
   const int cj = j >> 4, e = j & 15;
@@ -553,8 +598,17 @@ __device__ __forceinline__ float column_sum(float* red, int rg, int cc, const fl
   return __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
 }
 
-// fp64 deposit of the 16 pass-A partials (same swizzle idea, 16-byte chunks
-// of two doubles rotated by cc).
+// Deposit, barrier, total. The caller syncs before reusing `red`.
+template <int D>
+__device__ __forceinline__ float column_sum(float* red, int rg, int cc, const float2 (&part)[8]) {
+  column_deposit<D>(red, rg, cc, part);
+  __syncthreads();
+  return column_total<D>(red);
+}
+
+// fp64 deposit of the 8 partials of half `half` of a thread's 16 columns
+// (same swizzle idea: 16-byte chunks of two doubles rotated by cc), minus
+// the thread's per-row offsets.
 template <int D>
 __device__ __forceinline__ void deposit_f64(double* red, int rg, int cc, int half, const double (&acc)[8],
                                             double off) {
@@ -567,11 +621,11 @@ __device__ __forceinline__ void deposit_f64(double* red, int rg, int cc, int hal
 }
 
 // Column total of the fp64 partials, rounded once to fp32 (two threads per
-// column as in column_sum; column = threadIdx.x >> 1). Syncs first.
+// column as in column_total; column = threadIdx.x >> 1). The caller syncs
+// after the deposits.
 template <int D>
 __device__ __forceinline__ float column_total_f64(const double* red) {
   using G = Geo<D>;
-  __syncthreads();
   const int j = threadIdx.x >> 1;
   const int hh = threadIdx.x & 1;
   const int cj = j >> 4, e = j & 15;
@@ -586,7 +640,7 @@ __device__ __forceinline__ float column_total_f64(const double* red) {
   return __double2float_rn(a + __shfl_xor_sync(0xffffffffu, a, 1));
 }
 
-// ================================================================ step kernel
+// ================================================================ step kernels
 // Scalars of one tile, loaded by the producing thread one tile ahead of the
 // issue that needs them, so that their global-memory latency overlaps a
 // whole tile of compute.
@@ -615,9 +669,13 @@ __device__ __forceinline__ TileScalars load_scalars(const StepArgs& a, int tile,
   return x;
 }
 
+// ----------------------------------------------------------- FP32 state
+// The unquantized baseline: fp32 S in the pool, the same update rule in
+// fp32 (gate, S^T k, delta update, o), one tile per CTA iteration with the
+// tile held in registers.
 template <int D>
-__device__ __forceinline__ void issue_tile(const StepArgs& a, const TileScalars& x, uint8_t* stage_base,
-                                           uint64_t* bar, bool packed) {
+__device__ __forceinline__ void issue_fp32(const StepArgs& a, const TileScalars& x, uint8_t* stage_base,
+                                           uint64_t* bar) {
   Stage<D> s{stage_base, a.rec_cap};
   TileHdr* hd = s.hdr();
   if (x.slot < 0 || x.slot >= a.n_slots) {
@@ -629,39 +687,25 @@ __device__ __forceinline__ void issue_tile(const StepArgs& a, const TileScalars&
   const int hk = h / (a.h_v / a.h_k);
   const uint32_t vec = 4u * D;
   const bool kda = a.gate_kind != 0;
-  uint8_t* rec_src = packed ? a.pool + (uint64_t)x.slot * a.slot_bytes + x.rec_off
-                            : a.pool + ((uint64_t)x.slot * a.h_v + h) * (uint64_t)(4u * D * D);
+  uint8_t* rec_src = a.pool + ((uint64_t)x.slot * a.h_v + h) * (uint64_t)(4u * D * D);
   hd->dst = rec_src;
   hd->bytes = x.rec_bytes;
   hd->valid = 1;
   hd->beta = x.beta;
   hd->g = x.g;
-  hd->kind = x.kind;
-  uint32_t tx = x.rec_bytes + 3 * vec + (kda ? vec : 0u);
-  if (packed) tx += 3 * vec + 2u * D + (uint32_t)D;
+  hd->kind = 0;
+  const uint32_t tx = x.rec_bytes + 3 * vec + (kda ? vec : 0u);
   mbar_arrive_expect_tx(bar, tx);  // release: the header stores above become visible with the phase
   bulk_g2s(s.rec(), rec_src, x.rec_bytes, bar);
   bulk_g2s(s.k(), a.k + ((size_t)b * a.h_k + hk) * D, vec, bar);
   bulk_g2s(s.q(), a.q + ((size_t)b * a.h_k + hk) * D, vec, bar);
   bulk_g2s(s.v(), a.v + ((size_t)b * a.h_v + h) * D, vec, bar);
   if (kda) bulk_g2s(s.g(), a.g + ((size_t)b * a.h_v + h) * D, vec, bar);
-  if (packed) {
-    bulk_g2s(s.c(), a.t.col + (size_t)h * D, vec, bar);
-    bulk_g2s(s.ic(), a.t.icol + (size_t)h * D, vec, bar);
-    bulk_g2s(s.phi(), a.t.phi + (size_t)h * D, vec, bar);
-    bulk_g2s(s.row_off(), a.t.row_off + (size_t)h * D, 2u * D, bar);
-    bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
-  }
 }
 
-// The compute of one tile, from the stage in shared memory to the updated
-// record written back into the stage and o written to global memory. KC is
-// the width shared by every row of the head (ROW_PIVOT for an all-pivot
-// head), known at compile time, or 0 for heads whose rows differ (KDA):
-// with KC != 0 every per-row width switch folds away.
-template <int D, bool PACKED, int KC>
-__device__ __forceinline__ void tile_body(const StepArgs& a, const Stage<D>& S, const TileHdr& hd, float* red,
-                                          float* wsh, int* nf_sh, float* o, int rg, int cc, uint32_t& st) {
+template <int D>
+__device__ __forceinline__ void tile_body_fp32(const StepArgs& a, const Stage<D>& S, const TileHdr& hd, float* red,
+                                               float* wsh, float* o, int rg, int cc, uint32_t& st) {
   using G = Geo<D>;
   const int tid = threadIdx.x;
   const float* ks = S.k();
@@ -674,98 +718,29 @@ __device__ __forceinline__ void tile_body(const StepArgs& a, const Stage<D>& S, 
     qr[r] = qs[i];
     gr[r] = a.gate_kind == 0 ? hd.g : S.g()[i];
   }
-
-  // ---- pass A: values, gate, column sum S^T k
-  // packed: T holds the stored values V (codes or fp16) and mr the per-row
-  // multiplier M (a_i = r_i g_i, or g_i for a pivot row); the column sum
-  // is accumulated in fp64 from the exact per-row factors (see unpack_hi),
-  // in two halves of 8 columns to keep the accumulators few.
-  // fp32: T holds the gated state g_i S_ij and the column sum is fp32.
+  // gate and column sum S^T k
   float2 T[G::RPT][8];
-  float mr[G::RPT];
   float2 part[8];
-  float P;
-  if (PACKED) {
-    double kap[G::RPT];
-    double off = 0.0;
-    bool bad = false;
 #pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const int i = r * G::NG + rg;
-      const int code = KC ? KC : S.row_code()[i];
-      if (code == ROW_PIVOT) {
-        mr[r] = gr[r];
-        kap[r] = (double)gr[r] * (double)kr[r];
-      } else {
-        const float R = __half2float(reinterpret_cast<const __half*>(S.rec())[i]);
-        mr[r] = __fmul_rn(R, gr[r]);
-        const int E = code == 8 ? 12 : code;  // FieldPos<code>::E
-        kap[r] = (double)mr[r] * (double)kr[r] * (double)(1 << E);
-        off = off + (1.0 + (double)(1 << (code - 1)) / (double)(1 << E)) * kap[r];
-      }
-      bad |= !isfinite(mr[r]) || !isfinite(kr[r]);
+  for (int r = 0; r < G::RPT; ++r) {
+    const int i = r * G::NG + rg;
+    const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      float4 x = src[p];
+      T[r][2 * p] = __fmul2_rn(make_float2(x.x, x.y), f2(gr[r]));
+      T[r][2 * p + 1] = __fmul2_rn(make_float2(x.z, x.w), f2(gr[r]));
     }
-    double* red64 = reinterpret_cast<double*>(red);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      double acc[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-#pragma unroll
-      for (int r = 0; r < G::RPT; ++r) {
-        const int i = r * G::NG + rg;
-        const int code = KC ? KC : S.row_code()[i];
-        const uint8_t* row = S.rec() + row_offset<D, KC>(S.row_off(), i);
-        // unpack through temporaries: writing T[r] from inside the width
-        // switch would push the whole tile into local memory
-        float2 vt[8];
-        uint32_t xh[16];
-        unpack_hi(row, code, cc, vt, xh);
-#pragma unroll
-        for (int p = 0; p < 4; ++p) T[r][4 * half + p] = vt[4 * half + p];
-        if (code == ROW_PIVOT) {
-#pragma unroll
-          for (int p = 0; p < 4; ++p) bad |= !isfinite(vt[4 * half + p].x) || !isfinite(vt[4 * half + p].y);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[8 * half + j], 0), kap[r], acc[j]);
-      }
-      deposit_f64<D>(red64, rg, cc, half, acc, off);
-    }
-    if (bad) *nf_sh = 1;
-    P = column_total_f64<D>(red64);
-  } else {
-#pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const int i = r * G::NG + rg;
-      const float4* src = reinterpret_cast<const float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float4 x = src[p];
-        T[r][2 * p] = __fmul2_rn(make_float2(x.x, x.y), f2(gr[r]));
-        T[r][2 * p + 1] = __fmul2_rn(make_float2(x.z, x.w), f2(gr[r]));
-      }
-#pragma unroll
-      for (int p = 0; p < 8; ++p)
-        part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
-    }
-    P = column_sum<D>(red, rg, cc, part);
+    for (int p = 0; p < 8; ++p)
+      part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(kr[r])) : __ffma2_rn(T[r][p], f2(kr[r]), part[p]);
   }
+  const float P = column_sum<D>(red, rg, cc, part);
   if ((tid & 1) == 0) {
     const int j = tid >> 1;
-    float wj;
-    if (PACKED) {
-      const float p = __fmul_rn(S.c()[j], P);
-      const float u = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], p));
-      wj = __fmul_rn(u, S.ic()[j]);
-      if (!isfinite(wj)) *nf_sh = 1;
-    } else {
-      wj = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
-    }
-    wsh[j] = wj;
+    wsh[j] = __fmul_rn(hd.beta, __fsub_rn(S.v()[j], P));
   }
   __syncthreads();
-  const bool finite = *nf_sh == 0;
   float2 W[8];
   {
     const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
@@ -776,17 +751,12 @@ __device__ __forceinline__ void tile_body(const StepArgs& a, const Stage<D>& S, 
       W[2 * p + 1] = make_float2(x.z, x.w);
     }
   }
-  // ---- pass B: gate + delta update (one rounding), partial S^T q
+  // delta update, partial S^T q
 #pragma unroll
   for (int r = 0; r < G::RPT; ++r) {
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-      if (PACKED) {
-        const float2 kw = __fmul2_rn(f2(kr[r]), W[p]);
-        T[r][p] = __ffma2_rn(T[r][p], f2(mr[r]), kw);
-      } else {
-        T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
-      }
+      T[r][p] = __ffma2_rn(f2(kr[r]), W[p], T[r][p]);
       part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr[r])) : __ffma2_rn(T[r][p], f2(qr[r]), part[p]);
     }
   }
@@ -794,36 +764,28 @@ __device__ __forceinline__ void tile_body(const StepArgs& a, const Stage<D>& S, 
     const float O = column_sum<D>(red, rg, cc, part);
     if ((tid & 1) == 0) {
       const int j = tid >> 1;
-      const float oj = PACKED ? __fmul_rn(S.c()[j], O) : O;
-      if (oj != oj) st |= ST_NAN;
-      o[j] = oj;
+      if (O != O) st |= ST_NAN;
+      o[j] = O;
     }
   }
-  // ---- requantize (or store fp32) into the stage record, in place
-  if (PACKED) {
-    st |= requant_rows<D, KC>(S.rec(), S.row_off(), S.row_code(), S.phi(), rg, cc, finite, T);
-  } else {
 #pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const int i = r * G::NG + rg;
-      float4* dst = reinterpret_cast<float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
+  for (int r = 0; r < G::RPT; ++r) {
+    const int i = r * G::NG + rg;
+    float4* dst = reinterpret_cast<float4*>(S.rec() + ((size_t)i * D + 16 * cc) * 4);
 #pragma unroll
-      for (int p = 0; p < 4; ++p)
-        dst[p] = make_float4(T[r][2 * p].x, T[r][2 * p].y, T[r][2 * p + 1].x, T[r][2 * p + 1].y);
-    }
+    for (int p = 0; p < 4; ++p)
+      dst[p] = make_float4(T[r][2 * p].x, T[r][2 * p].y, T[r][2 * p + 1].x, T[r][2 * p + 1].y);
   }
 }
 
-// PACKED = true: quantized pool; false: fp32 S pool (unquantized baseline).
-template <int D, bool PACKED>
-__global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(const StepArgs a) {
+template <int D>
+__global__ void __launch_bounds__(Geo<D>::NT, 1) k_decode_step_fp32(const StepArgs a) {
   using G = Geo<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t bars[4];
   __shared__ __align__(16) float wsh[D];
   __shared__ uint32_t st_sh;
   __shared__ int abort_sh;
-  __shared__ int nf_sh;  // the current tile saw a non-finite input
   float* red = reinterpret_cast<float*>(smem + (size_t)a.nstage * a.stage_bytes);
 
   const int tid = threadIdx.x;
@@ -844,12 +806,11 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     fence_mbar_init();
     st_sh = 0;
     abort_sh = 0;
-    nf_sh = 0;
-    pre = load_scalars<D>(a, t0, t1, PACKED);
+    pre = load_scalars<D>(a, t0, t1, false);
     for (int s = 0; s < a.nstage && t0 + s < t1; ++s) {
       const TileScalars cur = pre;
-      pre = load_scalars<D>(a, t0 + s + 1, t1, PACKED);
-      issue_tile<D>(a, cur, smem + (size_t)s * a.stage_bytes, &bars[s], PACKED);
+      pre = load_scalars<D>(a, t0 + s + 1, t1, false);
+      issue_fp32<D>(a, cur, smem + (size_t)s * a.stage_bytes, &bars[s]);
     }
   }
   __syncthreads();
@@ -870,40 +831,24 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     const int h = tile - b * a.h_v;
     float* o = a.o + ((size_t)b * a.h_v + h) * D;
     const TileHdr hd = *S.hdr();
-    if (!hd.valid) {
-      if (tid < D) o[tid] = 0.0f;  // (nf_sh stays 0: nothing was computed)
+    if (hd.valid) {
+      tile_body_fp32<D>(a, S, hd, red, wsh, o, rg, cc, st);
+      fence_proxy_async_smem();
+    } else {
+      if (tid < D) o[tid] = 0.0f;
       st |= ST_SLOT;
-      // nothing was loaded into this stage; refill it if there is work left
-      __syncthreads();
-      if (tid == 0 && tile + a.nstage < t1) {
-        const TileScalars cur = pre;
-        pre = load_scalars<D>(a, tile + a.nstage + 1, t1, PACKED);
-        issue_tile<D>(a, cur, sbase, &bars[sidx], PACKED);
-      }
-      continue;
     }
-
-    switch (PACKED ? hd.kind : 0) {
-      case 8: tile_body<D, PACKED, (PACKED ? 8 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-      case 6: tile_body<D, PACKED, (PACKED ? 6 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-      case 4: tile_body<D, PACKED, (PACKED ? 4 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-      case 2: tile_body<D, PACKED, (PACKED ? 2 : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-      case ROW_PIVOT:
-        tile_body<D, PACKED, (PACKED ? ROW_PIVOT : 0)>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st);
-        break;
-      default: tile_body<D, PACKED, 0>(a, S, hd, red, wsh, &nf_sh, o, rg, cc, st); break;
-    }
-    fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      nf_sh = 0;  // every read of this tile's flag happened before the barrier above
-      bulk_s2g(hd.dst, S.rec(), hd.bytes);
-      bulk_commit();
-      bulk_wait_read_all();  // the stage may be refilled once the store has read it
+      if (hd.valid) {
+        bulk_s2g(hd.dst, S.rec(), hd.bytes);
+        bulk_commit();
+        bulk_wait_read_all();  // the stage may be refilled once the store has read it
+      }
       if (tile + a.nstage < t1) {
         const TileScalars cur = pre;
-        pre = load_scalars<D>(a, tile + a.nstage + 1, t1, PACKED);
-        issue_tile<D>(a, cur, sbase, &bars[sidx], PACKED);
+        pre = load_scalars<D>(a, tile + a.nstage + 1, t1, false);
+        issue_fp32<D>(a, cur, sbase, &bars[sidx]);
       }
     }
   }
@@ -913,6 +858,532 @@ __global__ void __launch_bounds__(Geo<D>::NT, PACKED ? 2 : 1) k_decode_step(cons
     if (abort_sh) {
       // give in-flight loads a bounded chance to land before the CTA exits
       for (int s = 0; s < a.nstage; ++s) (void)mbar_wait_bounded(&bars[s], 0, 1000000ull);
+    }
+    bulk_wait_all();
+    if (st_sh) atomicOr(a.t.status, st_sh);
+  }
+}
+
+// ----------------------------------------------------------- packed state
+// Per tile, three block barriers:
+//   wait for the stage; pass A: codes -> fp64 column partials of S^T k
+//   B1; column totals -> P, w = beta (v - c P) / c
+//   B2; pass B: codes read again -> T' = q a + k w (one rounding), o
+//       partials, row maxima, row scales, new codes written in place
+//   B3; o = c (column totals); thread 0 stores the record, and refills
+//       the stage right after the next tile's B1.
+// The partials of S^T k (fp64) and of S'^T q (fp32) share one buffer: a
+// thread deposits the next tile's S^T k partials only after every thread
+// has read this tile's o partials (an mbarrier every thread arrives on).
+
+// Control block of the producing thread (shared memory, thread 0 only).
+// The scalars of the next tile to issue are fetched with cp.async one
+// refill ahead (double-buffered by tile parity), so the producer never
+// waits on global memory in the middle of a tile.
+struct Producer {
+  int32_t slot[2];
+  uint32_t rec_off[2], rec_bytes[2];
+  uint32_t kind_word[2];  // the 4-byte word of head_kind holding the head's entry
+  float beta[2], g[2];
+  int next;  // next tile to issue
+  int pend;  // stage whose record store is issued and whose refill is pending, or -1
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Thread 0: start fetching the scalars of tile m (if it exists).
+__device__ __forceinline__ void prefetch_scalars(const StepArgs& a, Producer* pr, int m, int t1) {
+  if (m >= t1) return;
+  const int k = m & 1;
+  const int b = m / a.h_v;
+  const int h = m - b * a.h_v;
+  if (a.slots)
+    cp_async4(&pr->slot[k], a.slots + b);
+  else
+    pr->slot[k] = b;
+  cp_async4(&pr->rec_off[k], a.t.rec_off + h);
+  cp_async4(&pr->rec_bytes[k], a.t.rec_bytes + h);
+  cp_async4(&pr->kind_word[k], a.t.head_kind + (h & ~3));  // the table is padded to 16 bytes
+  cp_async4(&pr->beta[k], a.beta + m);
+  if (a.gate_kind == 0) cp_async4(&pr->g[k], a.g + m);
+  cp_async_commit();
+}
+
+// Issue tile x into a stage. All-pivot heads (kind ROW_PIVOT) are not
+// staged: their fp16 record is read and written in place in the pool, with
+// the L2 warmed by a bulk prefetch, so stages are sized for the largest
+// other record.
+template <int D>
+__device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalars& x, uint8_t* stage_base,
+                                             uint64_t* bar) {
+  Stage<D> s{stage_base, a.rec_cap};
+  TileHdr* hd = s.hdr();
+  if (x.slot < 0 || x.slot >= a.n_slots) {
+    hd->valid = 0;
+    mbar_arrive(bar);
+    return;
+  }
+  const int b = x.b, h = x.h;
+  const int hk = h / (a.h_v / a.h_k);
+  const uint32_t vec = 4u * D;
+  const bool kda = a.gate_kind != 0;
+  const bool direct = x.kind == ROW_PIVOT;
+  uint8_t* rec_src = a.pool + (uint64_t)x.slot * a.slot_bytes + x.rec_off;
+  hd->dst = rec_src;
+  hd->bytes = x.rec_bytes;
+  hd->valid = 1;
+  hd->beta = x.beta;
+  hd->g = x.g;
+  hd->kind = x.kind;
+  uint32_t tx = 6u * vec + (kda ? vec : 0u) + 3u * D;
+  if (!direct) tx += x.rec_bytes;
+  mbar_arrive_expect_tx(bar, tx);
+  if (direct)
+    bulk_prefetch_l2(rec_src, x.rec_bytes);
+  else
+    bulk_g2s(s.rec(), rec_src, x.rec_bytes, bar);
+  bulk_g2s(s.k(), a.k + ((size_t)b * a.h_k + hk) * D, vec, bar);
+  bulk_g2s(s.q(), a.q + ((size_t)b * a.h_k + hk) * D, vec, bar);
+  bulk_g2s(s.v(), a.v + ((size_t)b * a.h_v + h) * D, vec, bar);
+  if (kda) bulk_g2s(s.g(), a.g + ((size_t)b * a.h_v + h) * D, vec, bar);
+  bulk_g2s(s.c(), a.t.col + (size_t)h * D, vec, bar);
+  bulk_g2s(s.ic(), a.t.icol + (size_t)h * D, vec, bar);
+  bulk_g2s(s.phi(), a.t.phi + (size_t)h * D, vec, bar);
+  bulk_g2s(s.row_off(), a.t.row_off + (size_t)h * D, 2u * D, bar);
+  bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
+}
+
+// Thread 0: issue the next tile into stage s, then start fetching the
+// scalars of the one after it.
+template <int D>
+__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars, int t1,
+                                           int s) {
+  const int m = pr->next;
+  if (m >= t1) return;
+  cp_async_wait_all();
+  const int k = m & 1;
+  TileScalars x;
+  x.tile = m;
+  x.b = m / a.h_v;
+  x.h = m - x.b * a.h_v;
+  x.slot = pr->slot[k];
+  x.rec_off = pr->rec_off[k];
+  x.rec_bytes = pr->rec_bytes[k];
+  x.kind = (int)((pr->kind_word[k] >> (8 * (x.h & 3))) & 0xFFu);
+  x.beta = pr->beta[k];
+  x.g = a.gate_kind == 0 ? pr->g[k] : 0.0f;
+  pr->next = m + 1;
+  prefetch_scalars(a, pr, m + 1, t1);
+  issue_packed<D>(a, x, smem + (size_t)s * a.stage_bytes, &bars[s]);
+}
+
+// Thread 0: refill the stage whose store is pending, once the store has
+// read it (tiles go to stages round-robin, so the next tile to issue is
+// the one that belongs to that stage).
+template <int D>
+__device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars,
+                                               int t1) {
+  const int s = pr->pend;
+  if (s < 0) return;
+  pr->pend = -1;
+  bulk_wait_read_all();
+  issue_next<D>(a, pr, smem, bars, t1, s);
+}
+
+// Pass A, half H (8 columns) of a thread's chunk over its rows, for a head
+// of uniform width B (B = 16: all-pivot head, read from the pool when
+// DIRECT): the values go to T[r][4H..4H+3], the fp64 partials of S^T k to
+// acc. Only the words of half H are loaded.
+template <int D, int B, int H, bool DIRECT>
+__device__ __forceinline__ void pass_a_half(const uint8_t* rec, int rg, int cc, const double (&kap)[Geo<D>::RPT],
+                                            float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
+  uint32_t w[Geo<D>::RPT][B / 2];
+#pragma unroll
+  for (int r = 0; r < Geo<D>::RPT; ++r)
+    chunk_words<B, DIRECT>(rec + row_offset<D, B>(nullptr, r * Geo<D>::NG + rg), cc, w[r]);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+  for (int r = 0; r < Geo<D>::RPT; ++r) {
+    uint32_t xh[8];
+    float2 V[4];
+    if constexpr (B == 16)
+      hi_half_pivot<H>(w[r], xh, V);
+    else
+      hi_half_q<B, H>(w[r], xh, V);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) T[r][4 * H + p] = V[p];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap[r], acc[j]);
+  }
+}
+
+// Same for a head whose rows have different widths (one unit per key row).
+// The row's width decides the unpacking; values pass through temporaries
+// (writing T[r] inside the switch would send the tile to local memory).
+// Row offsets are clamped to the stage's record capacity: every read then
+// stays inside the stage even if its tables were never loaded (a wait that
+// gave up).
+template <int D, int H>
+__device__ __forceinline__ void pass_a_half_mixed(const uint8_t* rec, const uint16_t* row_off,
+                                                  const uint8_t* row_code, uint32_t rec_cap, int rg, int cc,
+                                                  const double (&kap)[Geo<D>::RPT], float2 (&T)[Geo<D>::RPT][8],
+                                                  double (&acc)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+#pragma unroll
+  for (int r = 0; r < Geo<D>::RPT; ++r) {
+    const int i = r * Geo<D>::NG + rg;
+    const uint8_t* row = rec + min((uint32_t)row_off[i], rec_cap);
+    uint32_t xh[8];
+    float2 V[4];
+    switch (row_code[i]) {
+      case 8: { uint32_t w[4]; chunk_words<8, false, false>(row, cc, w); hi_half_q<8, H>(w, xh, V); } break;
+      case 6: { uint32_t w[3]; chunk_words<6, false, false>(row, cc, w); hi_half_q<6, H>(w, xh, V); } break;
+      case 4: { uint32_t w[2]; chunk_words<4, false, false>(row, cc, w); hi_half_q<4, H>(w, xh, V); } break;
+      case 2: { uint32_t w[1]; chunk_words<2, false, false>(row, cc, w); hi_half_q<2, H>(w, xh, V); } break;
+      default: { uint32_t w[8]; chunk_words<16, false, false>(row, cc, w); hi_half_pivot<H>(w, xh, V); } break;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) T[r][4 * H + p] = V[p];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap[r], acc[j]);
+  }
+}
+
+// Requantization of RB rows (group grp of a thread's row slots): row maxima
+// over the LPR lanes of each row, one row scale per row (lane cc % RB of
+// the row group computes it, the others take it by shuffle), codes. Writes
+// the record (shared memory, or the pool for an all-pivot head). Pivot rows
+// keep their scale slot. `finite`: the tile's inputs were all finite, so no
+// T' is NaN and the plain maximum equals the NaN-propagating one.
+template <int D, int KC, int RB>
+__device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
+                                                  const float* phi, int grp, int rg, int cc, bool finite,
+                                                  const float2 (&T)[RB][8]) {
+  using G = Geo<D>;
+  uint32_t st = 0;
+  if constexpr (KC == ROW_PIVOT) {
+#pragma unroll
+    for (int u = 0; u < RB; ++u)
+      st |= store_row_pivot<true>(rec + row_offset<D, KC>(row_off, (grp * RB + u) * G::NG + rg), cc, T[u]);
+    return st;
+  } else {
+    float m[RB];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      float x = 0.0f;
+      if (finite) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) x = fmaxf(x, fmaxf(fabsf(T[u][p].x), fabsf(T[u][p].y)));
+#pragma unroll
+        for (int s = 1; s < G::LPR; s <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, s));
+      } else {
+#pragma unroll
+        for (int p = 0; p < 8; ++p) x = fmax_nan(x, fmax_nan(fabsf(T[u][p].x), fabsf(T[u][p].y)));
+#pragma unroll
+        for (int s = 1; s < G::LPR; s <<= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, s));
+      }
+      m[u] = x;
+    }
+    const int mine = cc % RB;
+    float mm = m[0];
+#pragma unroll
+    for (int u = 1; u < RB; ++u) mm = mine == u ? m[u] : mm;
+    const int im = (grp * RB + mine) * G::NG + rg;
+    const int cm = KC ? KC : row_code[im];
+    float ir_m = 0.0f;
+    uint16_t rbits = 0;
+    if (cm != ROW_PIVOT) {
+      if (mm != mm) {
+        st |= ST_NAN;
+      } else {
+        const float qm = (float)((1 << (cm - 1)) - 1);
+        const float s = __fdiv_rn(__fmul_rn(phi[im], mm), qm);
+        __half rh;
+        if (s > 65504.0f) {
+          rh = __ushort_as_half((unsigned short)0x7BFF);
+          st |= ST_SAT;
+        } else {
+          rh = __float2half_ru(s);
+        }
+        const float R = __half2float(rh);
+        ir_m = (R == 0.0f) ? 0.0f : __frcp_rn(R);
+        rbits = __half_as_ushort(rh);
+      }
+      if (cc < RB) reinterpret_cast<uint16_t*>(rec)[im] = rbits;
+    }
+    const int base = (int)(threadIdx.x & 31) - cc;
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
+      const int i = (grp * RB + u) * G::NG + rg;
+      const int code = KC ? KC : row_code[i];
+      uint8_t* row = rec + row_offset<D, KC>(row_off, i);
+      if (code == ROW_PIVOT) {
+        st |= store_row_pivot<false>(row, cc, T[u]);
+      } else if (m[u] != m[u]) {  // a NaN in the row: scale 0, all codes 0
+        store_row_zero(row, code, cc);
+      } else {
+        switch (code) {
+          case 8: store_row_q<8>(row, cc, ir, T[u]); break;
+          case 6: store_row_q<6>(row, cc, ir, T[u]); break;
+          case 4: store_row_q<4>(row, cc, ir, T[u]); break;
+          default: store_row_q<2>(row, cc, ir, T[u]); break;
+        }
+      }
+    }
+    return st;
+  }
+}
+
+// One tile of the packed step. KC is the width shared by every row of the
+// head (ROW_PIVOT: an all-pivot head, whose record stays in the pool), or 0
+// for heads whose rows differ; with KC != 0 every per-row width test folds
+// away. Returns false when a bounded wait gave up (the tile is abandoned).
+template <int D, int KC>
+__device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S, int sidx, uint32_t parity, int n,
+                                            uint64_t* bars, uint64_t* free_bar, uint8_t* smem, uint8_t* red,
+                                            float* wsh, float* msh, int* nf_sh, int* abort_sh, Producer* pr, int t1,
+                                            float* o, int rg, int cc, uint32_t& st) {
+  using G = Geo<D>;
+  constexpr bool DIRECT = KC == ROW_PIVOT;
+  const int tid = threadIdx.x;
+  const int base = (tid & 31) - cc;
+  const bool kda = a.gate_kind != 0;
+  const TileHdr* hd = S.hdr();
+  uint8_t* rec = DIRECT ? hd->dst : S.rec();
+  double* red64 = reinterpret_cast<double*>(red);
+
+  // ---- pass A: the tile's values into registers (T), fp64 column
+  // partials of S^T k
+  // A thread whose wait gave up still runs pass A, on stale but in-bounds
+  // shared memory, and the tile is abandoned at B1 before anything is
+  // written (keeping pass A unconditional keeps the tile in registers).
+  float2 T[G::RPT][8];
+  if (!mbar_wait_bounded(&bars[sidx], parity, 2000000000ull)) *abort_sh = 1;
+  {
+    // row factors: lane cc computes row slot cc % RPT, the others take it
+    // by shuffle. M = fp32(r g) (quantized row) or g (pivot row); the fp64
+    // weight kap = M k is exact.
+    const int mine = cc % G::RPT;
+    const int im = mine * G::NG + rg;
+    const int cm = KC ? KC : S.row_code()[im];
+    const float gm = kda ? S.g()[im] : hd->g;
+    const float mm =
+        cm == ROW_PIVOT ? gm : __fmul_rn(__half2float(reinterpret_cast<const __half*>(rec)[im]), gm);
+    if (cc < G::RPT) msh[im] = mm;
+    const double kapm = (double)mm * (double)S.k()[im];
+    double kap[G::RPT];
+    double off = 0.0;
+#pragma unroll
+    for (int r = 0; r < G::RPT; ++r) {
+      kap[r] = __shfl_sync(0xffffffffu, kapm, base + r);
+      const int code = KC ? KC : S.row_code()[r * G::NG + rg];
+      if (code != ROW_PIVOT) off = fma(code_offset(code), kap[r], off);
+    }
+    bool free_ok = true;
+    double acc[8];
+    if constexpr (KC != 0) {
+      pass_a_half<D, KC, 0, DIRECT>(rec, rg, cc, kap, T, acc);
+      // the buffer is free once every thread has read the previous tile's o partials
+      if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc, off);
+      pass_a_half<D, KC, 1, DIRECT>(rec, rg, cc, kap, T, acc);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc, off);
+    } else {
+      pass_a_half_mixed<D, 0>(rec, S.row_off(), S.row_code(), a.rec_cap, rg, cc, kap, T, acc);
+      if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc, off);
+      pass_a_half_mixed<D, 1>(rec, S.row_off(), S.row_code(), a.rec_cap, rg, cc, kap, T, acc);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc, off);
+    }
+    if (!free_ok) *abort_sh = 1;
+  }
+  __syncthreads();  // B1: the S^T k partials are complete
+  if (*abort_sh) return false;
+  if (tid == 0) refill_pending<D>(a, pr, smem, bars, t1);
+
+  // ---- column totals of S^T k -> w. A non-finite input anywhere in the
+  // tile (state, gate, k, v, beta) makes some w_j non-finite.
+  {
+    const float P = column_total_f64<D>(red64);
+    if ((tid & 1) == 0) {
+      const int j = tid >> 1;
+      const float p = __fmul_rn(S.c()[j], P);
+      const float u = __fmul_rn(hd->beta, __fsub_rn(S.v()[j], p));
+      const float wj = __fmul_rn(u, S.ic()[j]);
+      if (!isfinite(wj)) *nf_sh = 1;
+      wsh[j] = wj;
+    }
+  }
+  __syncthreads();  // B2: w is complete
+  const bool finite = *nf_sh == 0;
+
+  // ---- pass B: update (one rounding), o partials, requantization
+  float2 W[8];
+  {
+    const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float4 x = wsrc[p];
+      W[2 * p] = make_float2(x.x, x.y);
+      W[2 * p + 1] = make_float2(x.z, x.w);
+    }
+  }
+  float2 part[8];
+#pragma unroll
+  for (int r = 0; r < G::RPT; ++r) {
+    const int i = r * G::NG + rg;
+    const float kr = S.k()[i], qr = S.q()[i], M = msh[i];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      T[r][p] = __ffma2_rn(T[r][p], f2(M), __fmul2_rn(f2(kr), W[p]));
+      part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr)) : __ffma2_rn(T[r][p], f2(qr), part[p]);
+    }
+  }
+  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.phi(), 0, rg, cc, finite, T);
+  column_deposit<D>(reinterpret_cast<float*>(red), rg, cc, part);
+  if (!DIRECT) fence_proxy_async_smem();  // the new record is read by the bulk store
+  __syncthreads();  // B3: the o partials and the new record are complete
+
+  {
+    const float O = column_total<D>(reinterpret_cast<const float*>(red));
+    if ((tid & 1) == 0) {
+      const int j = tid >> 1;
+      const float oj = __fmul_rn(S.c()[j], O);
+      if (oj != oj) st |= ST_NAN;
+      o[j] = oj;
+    }
+  }
+  mbar_arrive(free_bar);  // this thread is done with the o partials
+  if (tid == 0) {
+    *nf_sh = 0;  // every read of this tile's flag happened before B3
+    if (!DIRECT) {
+      bulk_s2g(hd->dst, S.rec(), hd->bytes);
+      bulk_commit();
+    }
+    pr->pend = sidx;
+  }
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const StepArgs a) {
+  using G = Geo<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t bars[4];
+  __shared__ __align__(8) uint64_t free_bar;
+  __shared__ __align__(16) float wsh[D];
+  __shared__ __align__(16) float msh[D];
+  __shared__ Producer prod;
+  __shared__ uint32_t st_sh;
+  __shared__ int abort_sh;
+  __shared__ int nf_sh;  // the current tile saw a non-finite input
+  uint8_t* red = smem + (size_t)a.nstage * a.stage_bytes;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int cc = lane % G::LPR;
+  const int rg = warp * G::RPW + lane / G::LPR;
+
+  const int n_tiles = a.B * a.h_v;
+  const int per = (n_tiles + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * per;
+  const int t1 = min(n_tiles, t0 + per);
+  if (t0 >= t1) return;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.nstage; ++s) mbar_init(&bars[s], 1);
+    mbar_init(&free_bar, G::NT);
+    fence_mbar_init();
+    st_sh = 0;
+    abort_sh = 0;
+    nf_sh = 0;
+    prod.next = t0;
+    prod.pend = -1;
+    prefetch_scalars(a, &prod, t0, t1);
+    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, smem, bars, t1, s);
+  }
+  __syncthreads();
+
+  uint32_t st = 0;
+  int n = 0;
+  for (; t0 + n < t1; ++n) {
+    const int tile = t0 + n;
+    const int sidx = n % a.nstage;
+    const uint32_t parity = (uint32_t)(n / a.nstage) & 1u;
+    const Stage<D> S{smem + (size_t)sidx * a.stage_bytes, a.rec_cap};
+    const int b = tile / a.h_v;
+    const int h = tile - b * a.h_v;
+    float* o = a.o + ((size_t)b * a.h_v + h) * D;
+    // The header was written by thread 0 before at least one block barrier
+    // that every thread has passed since, so it is read without waiting for
+    // the stage's data; the dispatch below is uniform over the CTA.
+    if (!S.hdr()->valid) {
+      if (tid < D) o[tid] = 0.0f;
+      st |= ST_SLOT;
+      __syncthreads();  // every thread has read the header and finished the previous tile
+      mbar_arrive(&free_bar);
+      if (tid == 0) {
+        refill_pending<D>(a, &prod, smem, bars, t1);
+        prod.pend = sidx;  // nothing was loaded or stored: refill at the next refill point
+      }
+      __syncthreads();  // publish the refilled header before its tile is read
+      continue;
+    }
+    bool ok;
+    switch (S.hdr()->kind) {
+      case 8:
+        ok = packed_tile<D, 8>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+                               &prod, t1, o, rg, cc, st);
+        break;
+      case 6:
+        ok = packed_tile<D, 6>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+                               &prod, t1, o, rg, cc, st);
+        break;
+      case 4:
+        ok = packed_tile<D, 4>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+                               &prod, t1, o, rg, cc, st);
+        break;
+      case 2:
+        ok = packed_tile<D, 2>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+                               &prod, t1, o, rg, cc, st);
+        break;
+      case ROW_PIVOT:
+        ok = packed_tile<D, ROW_PIVOT>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh,
+                                       &abort_sh, &prod, t1, o, rg, cc, st);
+        break;
+      default:
+        ok = packed_tile<D, 0>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+                               &prod, t1, o, rg, cc, st);
+        break;
+    }
+    if (!ok) {
+      st |= ST_TIMEOUT;
+      break;
+    }
+  }
+  if (st) atomicOr(&st_sh, st);
+  __syncthreads();
+  if (tid == 0) {
+    if (abort_sh) {
+      // give the loads still in flight a bounded chance to land before the CTA exits
+      for (int m = t0 + n; m < prod.next; ++m) {
+        const int k = m - t0;
+        (void)mbar_wait_bounded(&bars[k % a.nstage], (uint32_t)(k / a.nstage) & 1u, 1000000ull);
+      }
     }
     bulk_wait_all();
     if (st_sh) atomicOr(a.t.status, st_sh);
