@@ -35,7 +35,10 @@
  *  - There is no CPU fallback: without a usable CUDA device every call that
  *    launches work returns SQ_ERR_CUDA.
  *  - Calls on one handle from different host threads must be serialized by
- *    the caller. Two steps in flight on the same pool slots race.
+ *    the caller. Two steps in flight on the same pool slots race. Steps of
+ *    one handle must also not run at the same time on the device (e.g. on
+ *    two unordered streams): they share the handle's work counter, which
+ *    each step leaves at zero when it ends.
  *
  * Storage format (SQ_FMT_PACKED). The pool is caller-owned device memory of
  * sq_state_bytes().pool_bytes bytes. Slot s starts at s * slot_bytes; in it

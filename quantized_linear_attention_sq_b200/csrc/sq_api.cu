@@ -37,6 +37,11 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 uint64_t round_up(uint64_t x, uint64_t m) { return (x + m - 1) / m * m; }
 
+// Tiles per scheduling chunk of the packed step: consecutive tiles of one
+// head run back to back on a CTA; the imbalance at the end is at most one
+// chunk per CTA.
+constexpr int kStepChunk = 2;
+
 }  // namespace
 
 struct sq_handle {
@@ -344,6 +349,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   h->tables.row_code = reinterpret_cast<const uint8_t*>(base + o_row_code);
   h->tables.head_kind = reinterpret_cast<const uint8_t*>(base + o_head_kind);
   h->tables.status = reinterpret_cast<uint32_t*>(base + o_status);
+  h->tables.sched = reinterpret_cast<uint32_t*>(base + o_status + 8);  // zero, and reset by every step launch
   s = plan_step(h);
   if (s != SQ_OK) {
     cudaFree(h->dev_block);
@@ -433,6 +439,7 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
   a.slots = slot_ids;
   a.B = B; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots; a.gate_kind = h->desc.gate;
   a.nstage = h->nstage; a.rec_cap = h->rec_cap; a.stage_bytes = h->stage_bytes;
+  a.chunk = kStepChunk;
   a.slot_bytes = h->slot_bytes;
   a.t = h->tables;
   const int n_tiles = B * h->desc.h_v;
@@ -704,6 +711,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.t.row_code = reinterpret_cast<const uint8_t*>(nd->scratch + o_row_code);
   a.t.head_kind = reinterpret_cast<const uint8_t*>(nd->scratch + o_head_kind);
   a.t.status = status ? status : reinterpret_cast<uint32_t*>(nd->scratch + o_status);
+  a.t.sched = reinterpret_cast<uint32_t*>(nd->scratch + o_status + 8);  // uploaded as zeros above
 
   // launch plan (same rule as a handle's)
   StepPlan p;
@@ -713,6 +721,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.rec_cap = p.rec_cap;
   a.stage_bytes = p.stage_bytes;
   a.nstage = p.nstage;
+  a.chunk = kStepChunk;
   const size_t smem = p.smem;
   const int blocks = p.blocks;
   const int n_tiles = B * hv;

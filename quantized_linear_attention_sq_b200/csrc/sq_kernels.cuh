@@ -47,6 +47,7 @@ struct Tables {
   const float* phi;           // [h_v*d] phi_i
   const uint8_t* head_kind;   // [h_v] width shared by all rows of the head (ROW_PIVOT: all pivot), 0: mixed
   uint32_t* status;           // device status word
+  uint32_t* sched;            // packed step: [0] next chunk of tiles, [1] CTAs done (both 0 between launches)
 };
 
 struct StepArgs {
@@ -60,6 +61,7 @@ struct StepArgs {
   const int32_t* slots; // [B] or null
   int32_t B, h_v, h_k, n_slots, gate_kind;
   int32_t nstage;
+  int32_t chunk;        // packed step: tiles per scheduling chunk
   uint32_t rec_cap;     // bytes reserved for a record in a stage (multiple of 128)
   uint32_t stage_bytes; // rec_cap + aux bytes, multiple of 128
   uint64_t slot_bytes;
@@ -174,7 +176,7 @@ struct TileHdr {
   float beta;
   float g;          // the head's gate (GDN); unused for KDA
   int32_t kind;     // width shared by every row of the head (ROW_PIVOT: all pivot), 0: mixed
-  uint32_t pad;
+  int32_t tile;     // packed step: b * h_v + h of the tile in this stage, or -1: no more tiles
 };
 
 // ------------------------------------------------------- code unpacking
@@ -876,16 +878,23 @@ __global__ void __launch_bounds__(Geo<D>::NT, 1) k_decode_step_fp32(const StepAr
 // thread deposits the next tile's S^T k partials only after every thread
 // has read this tile's o partials (an mbarrier every thread arrives on).
 
+// Tiles are numbered head-major, m = h B + b, and handed out in chunks of
+// a.chunk consecutive tiles from a global counter: a CTA works on one head
+// (one width, one code path) for several tiles in a row, and the CTAs stay
+// balanced although the widths cost differently.
+//
 // Control block of the producing thread (shared memory, thread 0 only).
 // The scalars of the next tile to issue are fetched with cp.async one
-// refill ahead (double-buffered by tile parity), so the producer never
-// waits on global memory in the middle of a tile.
+// refill ahead (double-buffered), and the next chunk is claimed one chunk
+// ahead, so the producer never waits on global memory inside a tile.
 struct Producer {
   int32_t slot[2];
   uint32_t rec_off[2], rec_bytes[2];
   uint32_t kind_word[2];  // the 4-byte word of head_kind holding the head's entry
   float beta[2], g[2];
-  int next;  // next tile to issue
+  int next;  // next tile to issue (head-major index), or -1: no more work
+  int end;   // end of the chunk that holds `next`
+  int buf;   // scalar buffer holding the scalars of `next`
   int pend;  // stage whose record store is issued and whose refill is pending, or -1
 };
 
@@ -901,12 +910,12 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Thread 0: start fetching the scalars of tile m (if it exists).
-__device__ __forceinline__ void prefetch_scalars(const StepArgs& a, Producer* pr, int m, int t1) {
-  if (m >= t1) return;
-  const int k = m & 1;
-  const int b = m / a.h_v;
-  const int h = m - b * a.h_v;
+// Thread 0: start fetching the scalars of tile m (head-major) into buffer k.
+__device__ __forceinline__ void prefetch_scalars(const StepArgs& a, Producer* pr, int m, int k) {
+  if (m < 0) return;
+  const int h = m / a.B;
+  const int b = m - h * a.B;
+  const int bh = b * a.h_v + h;
   if (a.slots)
     cp_async4(&pr->slot[k], a.slots + b);
   else
@@ -914,9 +923,27 @@ __device__ __forceinline__ void prefetch_scalars(const StepArgs& a, Producer* pr
   cp_async4(&pr->rec_off[k], a.t.rec_off + h);
   cp_async4(&pr->rec_bytes[k], a.t.rec_bytes + h);
   cp_async4(&pr->kind_word[k], a.t.head_kind + (h & ~3));  // the table is padded to 16 bytes
-  cp_async4(&pr->beta[k], a.beta + m);
-  if (a.gate_kind == 0) cp_async4(&pr->g[k], a.g + m);
+  cp_async4(&pr->beta[k], a.beta + bh);
+  if (a.gate_kind == 0) cp_async4(&pr->g[k], a.g + bh);
   cp_async_commit();
+}
+
+// Thread 0: set up the first chunk (the claim of the one after it, `ahead`,
+// is in flight when this returns).
+__device__ __forceinline__ void producer_start(const StepArgs& a, Producer* pr, int& ahead) {
+  const int n_tiles = a.B * a.h_v;
+  const int n_chunks = (n_tiles + a.chunk - 1) / a.chunk;
+  const int c0 = (int)atomicAdd(a.t.sched, 1u);
+  ahead = (int)atomicAdd(a.t.sched, 1u);
+  if (c0 < n_chunks) {
+    pr->next = c0 * a.chunk;
+    pr->end = min(pr->next + a.chunk, n_tiles);
+  } else {
+    pr->next = -1;
+  }
+  pr->buf = 0;
+  pr->pend = -1;
+  prefetch_scalars(a, pr, pr->next, 0);
 }
 
 // Issue tile x into a stage. All-pivot heads (kind ROW_PIVOT) are not
@@ -928,6 +955,7 @@ __device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalar
                                              uint64_t* bar) {
   Stage<D> s{stage_base, a.rec_cap};
   TileHdr* hd = s.hdr();
+  hd->tile = x.b * a.h_v + x.h;
   if (x.slot < 0 || x.slot >= a.n_slots) {
     hd->valid = 0;
     mbar_arrive(bar);
@@ -963,28 +991,47 @@ __device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalar
   bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
 }
 
-// Thread 0: issue the next tile into stage s, then start fetching the
-// scalars of the one after it.
+// Thread 0: issue the next tile into stage s (or mark the stage as the end
+// of the work), then start fetching the scalars of the tile after it,
+// claiming a new chunk when the current one is used up.
 template <int D>
-__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars, int t1,
-                                           int s) {
+__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars, int s,
+                                           int& ahead) {
+  uint8_t* base = smem + (size_t)s * a.stage_bytes;
   const int m = pr->next;
-  if (m >= t1) return;
+  if (m < 0) {
+    Stage<D>{base, a.rec_cap}.hdr()->tile = -1;
+    return;
+  }
   cp_async_wait_all();
-  const int k = m & 1;
+  const int k = pr->buf;
   TileScalars x;
-  x.tile = m;
-  x.b = m / a.h_v;
-  x.h = m - x.b * a.h_v;
+  x.h = m / a.B;
+  x.b = m - x.h * a.B;
+  x.tile = x.b * a.h_v + x.h;
   x.slot = pr->slot[k];
   x.rec_off = pr->rec_off[k];
   x.rec_bytes = pr->rec_bytes[k];
   x.kind = (int)((pr->kind_word[k] >> (8 * (x.h & 3))) & 0xFFu);
   x.beta = pr->beta[k];
   x.g = a.gate_kind == 0 ? pr->g[k] : 0.0f;
-  pr->next = m + 1;
-  prefetch_scalars(a, pr, m + 1, t1);
-  issue_packed<D>(a, x, smem + (size_t)s * a.stage_bytes, &bars[s]);
+  int nm = m + 1;
+  if (nm >= pr->end) {
+    const int n_tiles = a.B * a.h_v;
+    const int n_chunks = (n_tiles + a.chunk - 1) / a.chunk;
+    const int c = ahead;  // claimed a chunk ago
+    if (c < n_chunks) {
+      nm = c * a.chunk;
+      pr->end = min(nm + a.chunk, n_tiles);
+      ahead = (int)atomicAdd(a.t.sched, 1u);
+    } else {
+      nm = -1;
+    }
+  }
+  pr->next = nm;
+  pr->buf = k ^ 1;
+  prefetch_scalars(a, pr, nm, k ^ 1);
+  issue_packed<D>(a, x, base, &bars[s]);
 }
 
 // Thread 0: refill the stage whose store is pending, once the store has
@@ -992,12 +1039,12 @@ __device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint
 // the one that belongs to that stage).
 template <int D>
 __device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars,
-                                               int t1) {
+                                               int& ahead) {
   const int s = pr->pend;
   if (s < 0) return;
   pr->pend = -1;
   bulk_wait_read_all();
-  issue_next<D>(a, pr, smem, bars, t1, s);
+  issue_next<D>(a, pr, smem, bars, s, ahead);
 }
 
 // Pass A, half H (8 columns) of a thread's chunk over its rows, for a head
@@ -1154,8 +1201,8 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 template <int D, int KC>
 __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S, int sidx, uint32_t parity, int n,
                                             uint64_t* bars, uint64_t* free_bar, uint8_t* smem, uint8_t* red,
-                                            float* wsh, float* msh, int* nf_sh, int* abort_sh, Producer* pr, int t1,
-                                            float* o, int rg, int cc, uint32_t& st) {
+                                            float* wsh, float* msh, int* nf_sh, int* abort_sh, Producer* pr,
+                                            int& ahead, float* o, int rg, int cc, uint32_t& st) {
   using G = Geo<D>;
   constexpr bool DIRECT = KC == ROW_PIVOT;
   const int tid = threadIdx.x;
@@ -1212,7 +1259,7 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
   }
   __syncthreads();  // B1: the S^T k partials are complete
   if (*abort_sh) return false;
-  if (tid == 0) refill_pending<D>(a, pr, smem, bars, t1);
+  if (tid == 0) refill_pending<D>(a, pr, smem, bars, ahead);
 
   // ---- column totals of S^T k -> w. A non-finite input anywhere in the
   // tile (state, gate, k, v, beta) makes some w_j non-finite.
@@ -1298,12 +1345,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
   const int cc = lane % G::LPR;
   const int rg = warp * G::RPW + lane / G::LPR;
 
-  const int n_tiles = a.B * a.h_v;
-  const int per = (n_tiles + gridDim.x - 1) / gridDim.x;
-  const int t0 = blockIdx.x * per;
-  const int t1 = min(n_tiles, t0 + per);
-  if (t0 >= t1) return;
-
+  int ahead = 0;  // thread 0: the chunk claimed for after the current one
   if (tid == 0) {
     for (int s = 0; s < a.nstage; ++s) mbar_init(&bars[s], 1);
     mbar_init(&free_bar, G::NT);
@@ -1311,33 +1353,30 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
     st_sh = 0;
     abort_sh = 0;
     nf_sh = 0;
-    prod.next = t0;
-    prod.pend = -1;
-    prefetch_scalars(a, &prod, t0, t1);
-    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, smem, bars, t1, s);
+    producer_start(a, &prod, ahead);
+    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, smem, bars, s, ahead);
   }
   __syncthreads();
 
   uint32_t st = 0;
   int n = 0;
-  for (; t0 + n < t1; ++n) {
-    const int tile = t0 + n;
+  for (;; ++n) {
     const int sidx = n % a.nstage;
     const uint32_t parity = (uint32_t)(n / a.nstage) & 1u;
     const Stage<D> S{smem + (size_t)sidx * a.stage_bytes, a.rec_cap};
-    const int b = tile / a.h_v;
-    const int h = tile - b * a.h_v;
-    float* o = a.o + ((size_t)b * a.h_v + h) * D;
     // The header was written by thread 0 before at least one block barrier
     // that every thread has passed since, so it is read without waiting for
-    // the stage's data; the dispatch below is uniform over the CTA.
+    // the stage's data; the control flow below is uniform over the CTA.
+    const int tile = S.hdr()->tile;  // b * h_v + h
+    if (tile < 0) break;
+    float* o = a.o + (size_t)tile * D;
     if (!S.hdr()->valid) {
       if (tid < D) o[tid] = 0.0f;
       st |= ST_SLOT;
       __syncthreads();  // every thread has read the header and finished the previous tile
       mbar_arrive(&free_bar);
       if (tid == 0) {
-        refill_pending<D>(a, &prod, smem, bars, t1);
+        refill_pending<D>(a, &prod, smem, bars, ahead);
         prod.pend = sidx;  // nothing was loaded or stored: refill at the next refill point
       }
       __syncthreads();  // publish the refilled header before its tile is read
@@ -1347,27 +1386,27 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
     switch (S.hdr()->kind) {
       case 8:
         ok = packed_tile<D, 8>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
-                               &prod, t1, o, rg, cc, st);
+                               &prod, ahead, o, rg, cc, st);
         break;
       case 6:
         ok = packed_tile<D, 6>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
-                               &prod, t1, o, rg, cc, st);
+                               &prod, ahead, o, rg, cc, st);
         break;
       case 4:
         ok = packed_tile<D, 4>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
-                               &prod, t1, o, rg, cc, st);
+                               &prod, ahead, o, rg, cc, st);
         break;
       case 2:
         ok = packed_tile<D, 2>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
-                               &prod, t1, o, rg, cc, st);
+                               &prod, ahead, o, rg, cc, st);
         break;
       case ROW_PIVOT:
         ok = packed_tile<D, ROW_PIVOT>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh,
-                                       &abort_sh, &prod, t1, o, rg, cc, st);
+                                       &abort_sh, &prod, ahead, o, rg, cc, st);
         break;
       default:
         ok = packed_tile<D, 0>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
-                               &prod, t1, o, rg, cc, st);
+                               &prod, ahead, o, rg, cc, st);
         break;
     }
     if (!ok) {
@@ -1379,14 +1418,23 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
   __syncthreads();
   if (tid == 0) {
     if (abort_sh) {
-      // give the loads still in flight a bounded chance to land before the CTA exits
-      for (int m = t0 + n; m < prod.next; ++m) {
-        const int k = m - t0;
-        (void)mbar_wait_bounded(&bars[k % a.nstage], (uint32_t)(k / a.nstage) & 1u, 1000000ull);
+      // give the loads still in flight (tiles n .. n + nstage - 2) a bounded
+      // chance to land before the CTA exits
+      for (int k = 0; k + 1 < a.nstage; ++k) {
+        const TileHdr* hd = Stage<D>{smem + (size_t)((n + k) % a.nstage) * a.stage_bytes, a.rec_cap}.hdr();
+        if (hd->tile >= 0 && hd->valid)
+          (void)mbar_wait_bounded(&bars[(n + k) % a.nstage], (uint32_t)((n + k) / a.nstage) & 1u, 1000000ull);
       }
     }
     bulk_wait_all();
     if (st_sh) atomicOr(a.t.status, st_sh);
+    // The last CTA to finish resets the chunk counter for the next launch
+    // (every CTA's claims are ordered before its count by the fence).
+    __threadfence();
+    if (atomicAdd(a.t.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(a.t.sched, 0u);
+      atomicExch(a.t.sched + 1, 0u);
+    }
   }
 }
 
