@@ -142,19 +142,19 @@ struct Geo {
   static constexpr int NT = 32 * NW;          // threads per CTA
   static constexpr int NG = NW * RPW;         // row groups (= rows per pass of the CTA)
   static constexpr int RPT = D / NG;          // rows per thread
-  static constexpr int AUX = 31 * D + 32;     // aux bytes per stage (see stage layout)
+  static constexpr int AUX = (31 * D + 32 + 127) / 128 * 128;  // vector bytes per stage (see stage layout)
   static_assert(RPT >= 1 && RPT * NG == D, "bad geometry");
 };
 
-// Stage layout: [record: rec_cap][k f32 D][q f32 D][v f32 D][g f32 D]
-//               [c f32 D][ic f32 D][phi f32 D][row_off u16 D][row_code u8 D]
-//               [TileHdr 32 B]
+// Stage layout: [k f32 D][q f32 D][v f32 D][g f32 D][c f32 D][ic f32 D]
+//               [phi f32 D][row_off u16 D][row_code u8 D][TileHdr 32 B]
+//               (padded to Geo<D>::AUX bytes) [record: rec_cap]
+// Every offset but the stage's own base is a compile-time constant.
 template <int D>
 struct Stage {
   uint8_t* base;
   uint32_t rec_cap;
-  __device__ uint8_t* rec() const { return base; }
-  __device__ float* k() const { return reinterpret_cast<float*>(base + rec_cap); }
+  __device__ float* k() const { return reinterpret_cast<float*>(base); }
   __device__ float* q() const { return k() + D; }
   __device__ float* v() const { return k() + 2 * D; }
   __device__ float* g() const { return k() + 3 * D; }
@@ -164,6 +164,7 @@ struct Stage {
   __device__ uint16_t* row_off() const { return reinterpret_cast<uint16_t*>(k() + 7 * D); }
   __device__ uint8_t* row_code() const { return reinterpret_cast<uint8_t*>(row_off() + D); }
   __device__ struct TileHdr* hdr() const { return reinterpret_cast<struct TileHdr*>(row_code() + D); }
+  __device__ uint8_t* rec() const { return base + Geo<D>::AUX; }
 };
 
 // Per-tile scalars the producing thread writes next to the stage's data
@@ -590,14 +591,12 @@ __device__ __forceinline__ float column_total(const float* red) {
   const int hh = threadIdx.x & 1;
   const int cj = j >> 4, e = j & 15;
   const int off = 16 * cj + 4 * ((e >> 2) ^ ((cj >> 1) & 3)) + (e & 3);
-  float a0 = 0.f, a1 = 0.f;
+  // four independent partial sums keep the dependent chains short
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int g = 0; g < G::NG / 2; g += 2) {
-    a0 = __fadd_rn(a0, red[(hh * (G::NG / 2) + g) * D + off]);
-    a1 = __fadd_rn(a1, red[(hh * (G::NG / 2) + g + 1) * D + off]);
-  }
-  const float a = __fadd_rn(a0, a1);
-  return __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  for (int g = 0; g < G::NG / 2; ++g) a[g & 3] = __fadd_rn(a[g & 3], red[(hh * (G::NG / 2) + g) * D + off]);
+  const float t = __fadd_rn(__fadd_rn(a[0], a[1]), __fadd_rn(a[2], a[3]));
+  return __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 1));
 }
 
 // Deposit, barrier, total. The caller syncs before reusing `red`.
@@ -632,14 +631,11 @@ __device__ __forceinline__ float column_total_f64(const double* red) {
   const int hh = threadIdx.x & 1;
   const int cj = j >> 4, e = j & 15;
   const int off = 16 * cj + 2 * ((e >> 1) ^ (cj & 7)) + (e & 1);
-  double a0 = 0.0, a1 = 0.0;
+  double a[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-  for (int g = 0; g < G::NG / 2; g += 2) {
-    a0 += red[(hh * (G::NG / 2) + g) * D + off];
-    a1 += red[(hh * (G::NG / 2) + g + 1) * D + off];
-  }
-  const double a = a0 + a1;
-  return __double2float_rn(a + __shfl_xor_sync(0xffffffffu, a, 1));
+  for (int g = 0; g < G::NG / 2; ++g) a[g & 3] += red[(hh * (G::NG / 2) + g) * D + off];
+  const double t = (a[0] + a[1]) + (a[2] + a[3]);
+  return __double2float_rn(t + __shfl_xor_sync(0xffffffffu, t, 1));
 }
 
 // ================================================================ step kernels
@@ -995,9 +991,9 @@ __device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalar
 // of the work), then start fetching the scalars of the tile after it,
 // claiming a new chunk when the current one is used up.
 template <int D>
-__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars, int s,
+__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* stages, uint64_t* bars, int s,
                                            int& ahead) {
-  uint8_t* base = smem + (size_t)s * a.stage_bytes;
+  uint8_t* base = stages + (size_t)s * a.stage_bytes;
   const int m = pr->next;
   if (m < 0) {
     Stage<D>{base, a.rec_cap}.hdr()->tile = -1;
@@ -1038,13 +1034,13 @@ __device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint
 // read it (tiles go to stages round-robin, so the next tile to issue is
 // the one that belongs to that stage).
 template <int D>
-__device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, uint8_t* smem, uint64_t* bars,
+__device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, uint8_t* stages, uint64_t* bars,
                                                int& ahead) {
   const int s = pr->pend;
   if (s < 0) return;
   pr->pend = -1;
   bulk_wait_read_all();
-  issue_next<D>(a, pr, smem, bars, s, ahead);
+  issue_next<D>(a, pr, stages, bars, s, ahead);
 }
 
 // Pass A, half H (8 columns) of a thread's chunk over its rows, for a head
@@ -1108,15 +1104,40 @@ __device__ __forceinline__ void pass_a_half_mixed(const uint8_t* rec, const uint
   }
 }
 
+// max(|a|, |b|, |c|), NaN if any input is NaN (one instruction on sm_100).
+__device__ __forceinline__ float absmax3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max_j |T'_j| over the 16 values of a chunk (a depth-3 tree), then over
+// the LPR lanes of the row; NaN if any value of the row is NaN.
+template <int D>
+__device__ __forceinline__ float row_absmax(const float2 (&t)[8]) {
+  const float a0 = absmax3_nan(t[0].x, t[0].y, t[1].x);
+  const float a1 = absmax3_nan(t[1].y, t[2].x, t[2].y);
+  const float a2 = absmax3_nan(t[3].x, t[3].y, t[4].x);
+  const float a3 = absmax3_nan(t[4].y, t[5].x, t[5].y);
+  const float a4 = absmax3_nan(t[6].x, t[6].y, t[7].x);
+  const float b0 = absmax3_nan(a0, a1, a2);
+  const float b1 = absmax3_nan(a3, a4, t[7].y);
+  float x = fmax_nan(b0, b1);
+#pragma unroll
+  for (int s = 1; s < Geo<D>::LPR; s <<= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, s));
+  return x;
+}
+
 // Requantization of RB rows (group grp of a thread's row slots): row maxima
 // over the LPR lanes of each row, one row scale per row (lane cc % RB of
 // the row group computes it, the others take it by shuffle), codes. Writes
 // the record (shared memory, or the pool for an all-pivot head). Pivot rows
-// keep their scale slot. `finite`: the tile's inputs were all finite, so no
-// T' is NaN and the plain maximum equals the NaN-propagating one.
+// keep their scale slot. A row holding a NaN gets scale 0 and all codes 0;
+// such rows are found with one warp vote, so the common case runs without
+// per-row tests.
 template <int D, int KC, int RB>
 __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
-                                                  const float* phi, int grp, int rg, int cc, bool finite,
+                                                  const float* phi, int grp, int rg, int cc,
                                                   const float2 (&T)[RB][8]) {
   using G = Geo<D>;
   uint32_t st = 0;
@@ -1127,21 +1148,11 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
     return st;
   } else {
     float m[RB];
+    bool nan_row = false;
 #pragma unroll
     for (int u = 0; u < RB; ++u) {
-      float x = 0.0f;
-      if (finite) {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) x = fmaxf(x, fmaxf(fabsf(T[u][p].x), fabsf(T[u][p].y)));
-#pragma unroll
-        for (int s = 1; s < G::LPR; s <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, s));
-      } else {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) x = fmax_nan(x, fmax_nan(fabsf(T[u][p].x), fabsf(T[u][p].y)));
-#pragma unroll
-        for (int s = 1; s < G::LPR; s <<= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, s));
-      }
-      m[u] = x;
+      m[u] = row_absmax<D>(T[u]);
+      nan_row |= m[u] != m[u];
     }
     const int mine = cc % RB;
     float mm = m[0];
@@ -1150,11 +1161,9 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
     const int im = (grp * RB + mine) * G::NG + rg;
     const int cm = KC ? KC : row_code[im];
     float ir_m = 0.0f;
-    uint16_t rbits = 0;
     if (cm != ROW_PIVOT) {
-      if (mm != mm) {
-        st |= ST_NAN;
-      } else {
+      uint16_t rbits = 0;
+      if (mm == mm) {
         const float qm = (float)((1 << (cm - 1)) - 1);
         const float s = __fdiv_rn(__fmul_rn(phi[im], mm), qm);
         __half rh;
@@ -1171,22 +1180,40 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
       if (cc < RB) reinterpret_cast<uint16_t*>(rec)[im] = rbits;
     }
     const int base = (int)(threadIdx.x & 31) - cc;
+    if (!__any_sync(0xffffffffu, nan_row)) {
 #pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
-      const int i = (grp * RB + u) * G::NG + rg;
-      const int code = KC ? KC : row_code[i];
-      uint8_t* row = rec + row_offset<D, KC>(row_off, i);
-      if (code == ROW_PIVOT) {
-        st |= store_row_pivot<false>(row, cc, T[u]);
-      } else if (m[u] != m[u]) {  // a NaN in the row: scale 0, all codes 0
-        store_row_zero(row, code, cc);
-      } else {
+      for (int u = 0; u < RB; ++u) {
+        const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
+        const int i = (grp * RB + u) * G::NG + rg;
+        const int code = KC ? KC : row_code[i];
+        uint8_t* row = rec + row_offset<D, KC>(row_off, i);
         switch (code) {
           case 8: store_row_q<8>(row, cc, ir, T[u]); break;
           case 6: store_row_q<6>(row, cc, ir, T[u]); break;
           case 4: store_row_q<4>(row, cc, ir, T[u]); break;
-          default: store_row_q<2>(row, cc, ir, T[u]); break;
+          case 2: store_row_q<2>(row, cc, ir, T[u]); break;
+          default: st |= store_row_pivot<false>(row, cc, T[u]); break;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
+        const int i = (grp * RB + u) * G::NG + rg;
+        const int code = KC ? KC : row_code[i];
+        uint8_t* row = rec + row_offset<D, KC>(row_off, i);
+        if (code == ROW_PIVOT) {
+          st |= store_row_pivot<false>(row, cc, T[u]);
+        } else if (m[u] != m[u]) {
+          st |= ST_NAN;
+          store_row_zero(row, code, cc);
+        } else {
+          switch (code) {
+            case 8: store_row_q<8>(row, cc, ir, T[u]); break;
+            case 6: store_row_q<6>(row, cc, ir, T[u]); break;
+            case 4: store_row_q<4>(row, cc, ir, T[u]); break;
+            default: store_row_q<2>(row, cc, ir, T[u]); break;
+          }
         }
       }
     }
@@ -1200,8 +1227,8 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 // away. Returns false when a bounded wait gave up (the tile is abandoned).
 template <int D, int KC>
 __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S, int sidx, uint32_t parity, int n,
-                                            uint64_t* bars, uint64_t* free_bar, uint8_t* smem, uint8_t* red,
-                                            float* wsh, float* msh, int* nf_sh, int* abort_sh, Producer* pr,
+                                            uint64_t* bars, uint64_t* free_bar, uint8_t* stages, uint8_t* red,
+                                            float* wsh, float* msh, int* abort_sh, Producer* pr,
                                             int& ahead, float* o, int rg, int cc, uint32_t& st) {
   using G = Geo<D>;
   constexpr bool DIRECT = KC == ROW_PIVOT;
@@ -1259,23 +1286,19 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
   }
   __syncthreads();  // B1: the S^T k partials are complete
   if (*abort_sh) return false;
-  if (tid == 0) refill_pending<D>(a, pr, smem, bars, ahead);
+  if (tid == 0) refill_pending<D>(a, pr, stages, bars, ahead);
 
-  // ---- column totals of S^T k -> w. A non-finite input anywhere in the
-  // tile (state, gate, k, v, beta) makes some w_j non-finite.
+  // ---- column totals of S^T k -> w
   {
     const float P = column_total_f64<D>(red64);
     if ((tid & 1) == 0) {
       const int j = tid >> 1;
       const float p = __fmul_rn(S.c()[j], P);
       const float u = __fmul_rn(hd->beta, __fsub_rn(S.v()[j], p));
-      const float wj = __fmul_rn(u, S.ic()[j]);
-      if (!isfinite(wj)) *nf_sh = 1;
-      wsh[j] = wj;
+      wsh[j] = __fmul_rn(u, S.ic()[j]);
     }
   }
   __syncthreads();  // B2: w is complete
-  const bool finite = *nf_sh == 0;
 
   // ---- pass B: update (one rounding), o partials, requantization
   float2 W[8];
@@ -1299,7 +1322,7 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
       part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr)) : __ffma2_rn(T[r][p], f2(qr), part[p]);
     }
   }
-  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.phi(), 0, rg, cc, finite, T);
+  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.phi(), 0, rg, cc, T);
   column_deposit<D>(reinterpret_cast<float*>(red), rg, cc, part);
   if (!DIRECT) fence_proxy_async_smem();  // the new record is read by the bulk store
   __syncthreads();  // B3: the o partials and the new record are complete
@@ -1315,7 +1338,6 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
   }
   mbar_arrive(free_bar);  // this thread is done with the o partials
   if (tid == 0) {
-    *nf_sh = 0;  // every read of this tile's flag happened before B3
     if (!DIRECT) {
       bulk_s2g(hd->dst, S.rec(), hd->bytes);
       bulk_commit();
@@ -1336,8 +1358,9 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
   __shared__ Producer prod;
   __shared__ uint32_t st_sh;
   __shared__ int abort_sh;
-  __shared__ int nf_sh;  // the current tile saw a non-finite input
-  uint8_t* red = smem + (size_t)a.nstage * a.stage_bytes;
+  // [S^T k / o partials: NG D fp64][stage 0][stage 1]...
+  uint8_t* red = smem;
+  uint8_t* stages = smem + (size_t)G::NG * D * 8;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -1352,9 +1375,8 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
     fence_mbar_init();
     st_sh = 0;
     abort_sh = 0;
-    nf_sh = 0;
     producer_start(a, &prod, ahead);
-    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, smem, bars, s, ahead);
+    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, stages, bars, s, ahead);
   }
   __syncthreads();
 
@@ -1363,7 +1385,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
   for (;; ++n) {
     const int sidx = n % a.nstage;
     const uint32_t parity = (uint32_t)(n / a.nstage) & 1u;
-    const Stage<D> S{smem + (size_t)sidx * a.stage_bytes, a.rec_cap};
+    const Stage<D> S{stages + (size_t)sidx * a.stage_bytes, a.rec_cap};
     // The header was written by thread 0 before at least one block barrier
     // that every thread has passed since, so it is read without waiting for
     // the stage's data; the control flow below is uniform over the CTA.
@@ -1376,7 +1398,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
       __syncthreads();  // every thread has read the header and finished the previous tile
       mbar_arrive(&free_bar);
       if (tid == 0) {
-        refill_pending<D>(a, &prod, smem, bars, ahead);
+        refill_pending<D>(a, &prod, stages, bars, ahead);
         prod.pend = sidx;  // nothing was loaded or stored: refill at the next refill point
       }
       __syncthreads();  // publish the refilled header before its tile is read
@@ -1385,27 +1407,27 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
     bool ok;
     switch (S.hdr()->kind) {
       case 8:
-        ok = packed_tile<D, 8>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+        ok = packed_tile<D, 8>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
                                &prod, ahead, o, rg, cc, st);
         break;
       case 6:
-        ok = packed_tile<D, 6>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+        ok = packed_tile<D, 6>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
                                &prod, ahead, o, rg, cc, st);
         break;
       case 4:
-        ok = packed_tile<D, 4>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+        ok = packed_tile<D, 4>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
                                &prod, ahead, o, rg, cc, st);
         break;
       case 2:
-        ok = packed_tile<D, 2>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+        ok = packed_tile<D, 2>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
                                &prod, ahead, o, rg, cc, st);
         break;
       case ROW_PIVOT:
-        ok = packed_tile<D, ROW_PIVOT>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh,
+        ok = packed_tile<D, ROW_PIVOT>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh,
                                        &abort_sh, &prod, ahead, o, rg, cc, st);
         break;
       default:
-        ok = packed_tile<D, 0>(a, S, sidx, parity, n, bars, &free_bar, smem, red, wsh, msh, &nf_sh, &abort_sh,
+        ok = packed_tile<D, 0>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
                                &prod, ahead, o, rg, cc, st);
         break;
     }
@@ -1421,7 +1443,7 @@ __global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const Step
       // give the loads still in flight (tiles n .. n + nstage - 2) a bounded
       // chance to land before the CTA exits
       for (int k = 0; k + 1 < a.nstage; ++k) {
-        const TileHdr* hd = Stage<D>{smem + (size_t)((n + k) % a.nstage) * a.stage_bytes, a.rec_cap}.hdr();
+        const TileHdr* hd = Stage<D>{stages + (size_t)((n + k) % a.nstage) * a.stage_bytes, a.rec_cap}.hdr();
         if (hd->tile >= 0 && hd->valid)
           (void)mbar_wait_bounded(&bars[(n + k) % a.nstage], (uint32_t)((n + k) / a.nstage) & 1u, 1000000ull);
       }
