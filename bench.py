@@ -250,8 +250,8 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "kernel": "k_decode_step<128,packed>", "algorithmic_bytes_per_launch": bytes_launch,
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "kernel": "k_decode_step_packed<128>", "algorithmic_bytes_per_launch": bytes_launch,
                      "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
                   "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
@@ -263,7 +263,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args, sample_requests=args.cpu_sample_requests)
+        out["cpu_baseline"] = cpu_baseline(args, target_s=args.cpu_seconds)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -273,30 +273,63 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(out), flush=True)
 
 
+def profiled_traffic():
+    """DRAM bytes (read + write) per launch of the packed step from the ncu
+    capture recorded under profiles/, or None once the kernel source has
+    changed since that capture."""
+    import hashlib
+    rec_path = os.path.join(ROOT, "profiles", "k_decode_step_packed_gdn_serving_b512.traffic.json")
+    try:
+        rec = json.load(open(rec_path))
+        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+    except (OSError, ValueError, KeyError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec["kernel_source_sha256"]:
+        return None
+    return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
 # ------------------------------------------------------- the CPU oracle
-def cpu_baseline(args, sample_requests=64, steps=None):
-    """Time the CPU oracle (as it stands) on a bounded sample of the workload:
-    `sample_requests` requests x 32 heads, `steps` decode steps, tiles split
-    over all host cores."""
+def cpu_baseline(args, target_s=15.0, steps=None):
+    """Time the CPU oracle (as it stands) on a bounded sample of the
+    workload, tiles split over all host cores: a short probe measures the
+    oracle's rate on this host, then `steps` decode steps (default: as many
+    as fit) on as many of the batch's requests as make the timed part last
+    about `target_s` seconds."""
     import oracle
     from quantized_linear_attention_sq_b200 import synth
 
     w = synth.workload(CONFIG_ID, seed=args.seed)
     c = w.cfg
     cal = w.calib()
-    reqs = list(range(sample_requests))
-    o_ = oracle.Oracle(len(reqs), c.h_v, c.h_k, c.d, c.gate_kind, cal.unit_bits, cal.pivot, cal.col_scale,
-                       cal.row_impact)
-    pool = o_.new_pool()
-    S = w.initial_state(reqs)
-    S *= w.outlier_mask()[None, :, None, :]
-    o_.quantize(pool, S)
     cores = oracle.cores_available()
-    steps = steps or args.cpu_steps
-    inputs = [w.step_inputs(t, reqs) for t in range(steps)]
+
+    def setup(reqs):
+        o_ = oracle.Oracle(len(reqs), c.h_v, c.h_k, c.d, c.gate_kind, cal.unit_bits, cal.pivot, cal.col_scale,
+                           cal.row_impact)
+        pool = o_.new_pool()
+        S = w.initial_state(reqs)
+        S *= w.outlier_mask()[None, :, None, :]
+        o_.quantize(pool, S)
+        return o_, pool
+
+    # probe: one step on a few requests gives the tile-steps per second
+    probe = list(range(min(c.batch, 2 * cores)))
+    o_, pool = setup(probe)
+    x = w.step_inputs(0, probe)
+    t0 = time.perf_counter()
+    o_.step(pool, *x, threads=cores)
+    rate = len(probe) * c.h_v / max(time.perf_counter() - t0, 1e-6)
+    budget = rate * target_s  # tile-steps
+    if steps is None:
+        steps = max(1, min(64, int(budget // (c.batch * c.h_v))))
+    n_req = max(1, min(c.batch, int(budget // (steps * c.h_v))))
+    reqs = list(range(n_req))
+    o_, pool = setup(reqs)
+    inputs = [w.step_inputs(t, reqs) for t in range(min(steps, 8))]
     t0 = time.perf_counter()
     for t in range(steps):
-        o_.step(pool, *inputs[t], threads=cores)
+        o_.step(pool, *inputs[t % len(inputs)], threads=cores)
     dt = time.perf_counter() - t0
     units = len(reqs) * c.h_v * steps
     return {"value": units / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -307,7 +340,9 @@ def cpu_baseline(args, sample_requests=64, steps=None):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    cb = cpu_baseline(args, sample_requests=args.cpu_sample_requests, steps=max(1, args.steps))
+    # each of the --steps steps is a bounded sample of the workload; the whole
+    # run is sized to about a minute of CPU time
+    cb = cpu_baseline(args, target_s=60.0, steps=max(1, args.steps))
     from quantized_linear_attention_sq_b200 import synth
     w = synth.workload(CONFIG_ID, seed=args.seed)
     out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
@@ -327,8 +362,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-requests", type=int, default=48)
-    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--profile", type=int, default=0,
                     help="prepare the workload, run this many packed steps untimed, exit (for ncu)")
     args = ap.parse_args()
