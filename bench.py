@@ -113,7 +113,7 @@ class ClockSampler:
 # --------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
-    from quantized_linear_attention_sq_b200 import _abi, build, synth
+    from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
     from quantized_linear_attention_sq_b200.state import StatePool
 
     torch.cuda.set_device(local_rank)
@@ -123,7 +123,7 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = synth.workload(CONFIG_ID, seed=args.seed + rank)   # each rank: its own 512 requests
+    w = synth.workload(CONFIG_ID, seed=shards.rank_seed(args.seed, rank))   # each rank: its own 512 requests
     c = w.cfg
     cal = w.calib()
     B = c.batch
@@ -166,11 +166,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return shards.max_over_ranks(x, dist, dev)
 
     # ---- device-resident timing (per-launch events on the launching stream)
     def timed_device(spool, pl, K, W):
@@ -235,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
     rep = sp.report
     frep = fp.report
     units = B * c.h_v
-    value = world * units * args.steps / (total_ms / 1e3)
+    value = shards.job_rate(units, args.steps, total_ms, world)
     bytes_launch = B * rep["state_bytes_per_step"]
     peak, peak_kind = peaks()
     achieved = bytes_launch / (kern_ms / 1e3) / 1e9
@@ -246,7 +242,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
         "config": workload_config(w),
-        "e2e": {"value": world * units * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": shards.job_rate(units, args.steps, e2e_ms, world), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -256,7 +252,7 @@ def run_ours(args, rank, world, local_rank):
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
                   "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
                   "status_bits": st_bits},
-        "fp32_state": {"value": world * units * max(4, args.steps // 4) / (fp_total / 1e3),
+        "fp32_state": {"value": shards.job_rate(units, max(4, args.steps // 4), fp_total, world),
                        "kernel_ms": fp_kern, "achieved_gbs": fp_bytes / (fp_kern / 1e3) / 1e9,
                        "frac": fp_bytes / (fp_kern / 1e3) / 1e9 / peak,
                        "speedup_quantized_vs_fp32": fp_kern / kern_ms},
