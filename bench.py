@@ -143,6 +143,7 @@ def run_ours(args, rank, world, local_rank):
     S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
     sp = make(_abi.SQ_FMT_PACKED)
     pool = sp.new_pool()
+    clip = clip_fraction(S, cal, c)
     sp.quantize_state(pool, S)
     torch.cuda.synchronize()
     setup_status = sp.get_status()
@@ -250,6 +251,7 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "k_decode_step_packed<128>", "algorithmic_bytes_per_launch": bytes_launch,
                      "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
+                  "clip_fraction": clip,
                   "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
                   "status_bits": st_bits},
         "fp32_state": {"value": shards.job_rate(units, max(4, args.steps // 4), fp_total, world),
@@ -283,6 +285,37 @@ def profiled_traffic():
     if hashlib.sha256(src).hexdigest() != rec["kernel_source_sha256"]:
         return None
     return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+
+
+def clip_fraction(S, cal, c):
+    """Share of the quantized rows' entries that the row scale clips when
+    the state S [B, h_v, d, d] is quantized: |T_ij| / r_i rounds beyond qmax,
+    with T = S / c and r_i the fp16 round-up of phi_i max_j |T_ij| / qmax
+    (rows with phi_i < 1 clip their largest entries). GDN units (one width
+    per head); pivot heads are not counted."""
+    import torch
+
+    dev = S.device
+    keep = torch.from_numpy(cal.pivot == 0).to(dev)                           # [h_v]
+    qmax = torch.from_numpy((2.0 ** (cal.unit_bits.astype("float64") - 1) - 1).astype("float32")).to(dev)
+    ic = 1.0 / torch.from_numpy(cal.col_scale).to(dev)                         # [h_v, d]
+    phi = torch.from_numpy(cal.row_impact).to(dev)                             # [h_v, d]
+    clipped = 0
+    total = 0
+    for b0 in range(0, S.shape[0], 64):                                        # bounded temporaries
+        T = S[b0:b0 + 64] * ic[None, :, None, :]
+        m = T.abs().amax(dim=3)                                                # [b, h_v, d]
+        s = phi[None] * m / qmax[None, :, None]
+        h = s.to(torch.float16)
+        up = (h.float() < s) & (h.float() < 65504)
+        h = torch.where(up, (h.view(torch.int16) + 1).view(torch.float16), h)   # round toward +inf
+        r = h.float()
+        lim = qmax[None, :, None, None] + 0.5
+        over = (T.abs() * (1.0 / r).unsqueeze(3)) > lim
+        over = over & keep[None, :, None, None] & (r > 0).unsqueeze(3)
+        clipped += int(over.sum())
+        total += int(keep.sum()) * T.shape[0] * c.d * c.d
+    return clipped / max(total, 1)
 
 
 # ------------------------------------------------------- the CPU oracle
@@ -350,12 +383,101 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------- 8-layer KDA rollout (CUDA graph)
+def run_rollout(args, rank, world, local_rank):
+    """The long-rollout workload (8 KDA layers, 256 requests x 32 heads per
+    GPU, widths {2,4,6} at 4-bit nominal): one token = one step of every
+    layer. Timed with per-layer launches and with one CUDA graph holding 4
+    tokens x 8 layers of launches (prints its own JSON line)."""
+    import torch
+    from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
+    from quantized_linear_attention_sq_b200.rollout import LayerStack
+    from quantized_linear_attention_sq_b200.state import StatePool
+
+    torch.cuda.set_device(local_rank)
+    build.build()
+    dev = torch.device("cuda", local_rank)
+    cid = 4
+    nl = synth.CONFIGS[cid].layers
+    works = [synth.workload(cid, seed=shards.rank_seed(args.seed, rank), layer=l) for l in range(nl)]
+    c = works[0].cfg
+    B = c.batch
+    layers, pools = [], []
+    for w in works:
+        cal = w.calib()
+        fp = StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, _abi.SQ_FMT_FP32)
+        S = torch.from_numpy(w.initial_state()).to(dev)
+        o = torch.empty((B, c.h_v, c.d), device=dev)
+        for t in range(-c.warmup_steps, 0):
+            fp.decode_step(S, *(torch.from_numpy(x).to(dev) for x in w.step_inputs(t)), o)
+        S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
+        sp = StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, _abi.SQ_FMT_PACKED, cal.unit_bits, cal.pivot,
+                       cal.col_scale, cal.row_impact)
+        pool = sp.new_pool()
+        sp.quantize_state(pool, S)
+        torch.cuda.synchronize()
+        del S
+        fp.close()
+        layers.append(sp)
+        pools.append(pool)
+    stack = LayerStack(layers)
+    NI = 4
+    inputs = [[[torch.from_numpy(x).to(dev) for x in w.step_inputs(t)] for w in works] for t in range(NI)]
+    outs = [[torch.empty((B, c.h_v, c.d), device=dev) for _ in works] for _ in range(NI)]
+    K = max(NI, args.steps // NI * NI)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def eager_block():
+        for t in range(NI):
+            stack.step(pools, inputs[t], outs[t])
+
+    eager_ms = timed(eager_block, K // NI)
+    graph = stack.capture(pools, inputs, outs)
+    graph_ms = timed(graph.replay, K // NI)
+    status = [sp.get_status() for sp in layers]
+    units = B * c.h_v * nl
+    bytes_token = sum(B * sp.report["state_bytes_per_step"] for sp in layers)
+    peak, peak_kind = peaks()
+    out = {"metric": "8-layer KDA rollout (request*head*layer)-steps/s", "unit": "(request*head*layer)-steps/s",
+           "n_gpus": world, "tokens": K, "warmup_blocks": args.warmup,
+           "config": {"workload": c.name, "batch_per_gpu": B, "h_v": c.h_v, "d": c.d, "layers": nl,
+                      "gate": "KDA (one gate per key channel)",
+                      "widths": "per-row {2,4,6}, 4-bit nominal, 3% FP16 pivot rows"},
+           "eager": {"value": units * K / (eager_ms / 1e3), "ms_per_token": eager_ms / K,
+                     "launches_per_token": nl},
+           "graph": {"value": units * K / (graph_ms / 1e3), "ms_per_token": graph_ms / K,
+                     "tokens_per_replay": NI, "launches_per_replay": NI * nl},
+           "graph_speedup": eager_ms / graph_ms,
+           "achieved_gbs_graph": bytes_token / (graph_ms / K / 1e3) / 1e9,
+           "frac_graph": bytes_token / (graph_ms / K / 1e3) / 1e9 / peak,
+           "peak_kind": f"{peak_kind} hbm_gbs (copy)", "status_bits": status}
+    del graph
+    stack.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers"], default="serving",
+                    help="serving: the headline GDN workload; kda_rollout_8layers: 8 KDA layers, "
+                         "per-layer launches vs one CUDA graph")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -370,6 +492,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "kda_rollout_8layers":
+        run_rollout(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -177,7 +177,7 @@ uint64_t sq_launch_count(const sq_handle* h);
  * it out for the same `desc` and `calib`, but without a handle:
  *   - the per-head tables (record and row offsets, widths, c, 1/c, phi)
  *     are rebuilt on the host from `calib` at every call and copied into a
- *     fixed 128 KiB array in device memory that this library declares at
+ *     fixed 160 KiB array in device memory that this library declares at
  *     file scope (every GPU that loads the library holds it until the
  *     process exits); nothing is allocated on the device or the host heap;
  *   - limits: packed pools only, h_v <= SQ_NOALLOC_MAX_HEADS, and the tables

@@ -136,7 +136,7 @@ sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int o
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
   const size_t static_smem = fa.sharedSizeBytes;
   p->rec_cap = (uint32_t)round_up(stage_rec < 16 ? 16 : stage_rec, 128);
-  p->stage_bytes = (uint32_t)round_up(p->rec_cap + 31u * d + 32u, 128);  // + vectors, tables, header
+  p->stage_bytes = (uint32_t)round_up(p->rec_cap + 32u * d + 32u, 128);  // + vectors, tables, header
   const int NG = 32;  // row groups per CTA: 32 for every supported d
   const size_t red = (size_t)NG * d * (packed ? 8 : 4);
   const size_t dyn_max = (size_t)optin_smem - static_smem;
@@ -165,6 +165,23 @@ sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int o
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
   if (p->blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
   return SQ_OK;
+}
+
+// Thread-slot order of a head's rows for the packed step: the identity for a
+// head of uniform width; for a head whose rows differ, the rows grouped by
+// width (stable), so the rows a warp handles together share one code path.
+void build_row_perm(const uint8_t* row_code, int d, uint8_t* perm) {
+  bool uniform = true;
+  for (int i = 1; i < d; ++i) uniform = uniform && row_code[i] == row_code[0];
+  int s = 0;
+  if (uniform) {
+    for (int i = 0; i < d; ++i) perm[i] = (uint8_t)i;
+    return;
+  }
+  const uint8_t order[5] = {2, 4, 6, 8, sqk::ROW_PIVOT};
+  for (uint8_t code : order)
+    for (int i = 0; i < d; ++i)
+      if (row_code[i] == code) perm[s++] = (uint8_t)i;
 }
 
 // Largest record that goes through a stage: that of every head except the
@@ -303,7 +320,8 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   size_t o_phi = round_up(o_icol + 4 * nhd, 16);
   size_t o_row_off = round_up(o_phi + 4 * nhd, 16);
   size_t o_row_code = round_up(o_row_off + 2 * nhd, 16);
-  size_t o_head_kind = round_up(o_row_code + nhd, 16);
+  size_t o_row_perm = round_up(o_row_code + nhd, 16);
+  size_t o_head_kind = round_up(o_row_perm + nhd, 16);
   size_t o_status = round_up(o_head_kind + hv, 16);
   size_t total = round_up(o_status + 16, 256);
   std::vector<uint8_t> host(total, 0);
@@ -320,6 +338,8 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   }
   memcpy(host.data() + o_row_off, h->row_off.data(), 2 * nhd);
   memcpy(host.data() + o_row_code, h->row_code.data(), nhd);
+  for (int hh = 0; hh < hv; ++hh)
+    build_row_perm(h->row_code.data() + (size_t)hh * d, d, host.data() + o_row_perm + (size_t)hh * d);
   for (int hh = 0; hh < hv; ++hh) {  // width shared by every row of the head, else 0
     uint8_t k = packed ? h->row_code[(size_t)hh * d] : 0;
     for (int i = 1; i < d && k; ++i)
@@ -347,6 +367,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   h->tables.phi = reinterpret_cast<const float*>(base + o_phi);
   h->tables.row_off = reinterpret_cast<const uint16_t*>(base + o_row_off);
   h->tables.row_code = reinterpret_cast<const uint8_t*>(base + o_row_code);
+  h->tables.row_perm = reinterpret_cast<const uint8_t*>(base + o_row_perm);
   h->tables.head_kind = reinterpret_cast<const uint8_t*>(base + o_head_kind);
   h->tables.status = reinterpret_cast<uint32_t*>(base + o_status);
   h->tables.sched = reinterpret_cast<uint32_t*>(base + o_status + 8);  // zero, and reset by every step launch
@@ -546,7 +567,7 @@ sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, cons
 // ===================================================================
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 128 * 1024;
+constexpr size_t kNoAllocScratchBytes = 160 * 1024;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Host staging for the tables (the copy from pageable memory returns only
@@ -640,7 +661,8 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   const size_t o_phi = round_up(o_icol + 4 * nhd, 16);
   const size_t o_row_off = round_up(o_phi + 4 * nhd, 16);
   const size_t o_row_code = round_up(o_row_off + 2 * nhd, 16);
-  const size_t o_head_kind = round_up(o_row_code + nhd, 16);
+  const size_t o_row_perm = round_up(o_row_code + nhd, 16);
+  const size_t o_head_kind = round_up(o_row_perm + nhd, 16);
   const size_t o_status = round_up(o_head_kind + (size_t)hv, 16);
   const size_t total = round_up(o_status + 16, 16);
   if (total > kNoAllocScratchBytes)
@@ -685,6 +707,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
     for (int i = 1; i < d && kind; ++i)
       if (row_code[(size_t)hh * d + i] != kind) kind = 0;
     head_kind[hh] = kind;
+    build_row_perm(row_code + (size_t)hh * d, d, host + o_row_perm + (size_t)hh * d);
   }
   for (size_t x = 0; x < nhd; ++x) {
     col[x] = calib->col_scale[x];
@@ -709,6 +732,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.t.phi = reinterpret_cast<const float*>(nd->scratch + o_phi);
   a.t.row_off = reinterpret_cast<const uint16_t*>(nd->scratch + o_row_off);
   a.t.row_code = reinterpret_cast<const uint8_t*>(nd->scratch + o_row_code);
+  a.t.row_perm = reinterpret_cast<const uint8_t*>(nd->scratch + o_row_perm);
   a.t.head_kind = reinterpret_cast<const uint8_t*>(nd->scratch + o_head_kind);
   a.t.status = status ? status : reinterpret_cast<uint32_t*>(nd->scratch + o_status);
   a.t.sched = reinterpret_cast<uint32_t*>(nd->scratch + o_status + 8);  // uploaded as zeros above

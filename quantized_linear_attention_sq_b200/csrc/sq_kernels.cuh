@@ -42,6 +42,8 @@ struct Tables {
   const uint32_t* rec_bytes;  // [h_v] record size (multiple of 16)
   const uint16_t* row_off;    // [h_v*d] byte offset of key row i inside the record
   const uint8_t* row_code;    // [h_v*d] 2, 4, 6, 8 or ROW_PIVOT
+  const uint8_t* row_perm;    // [h_v*d] packed step: row held in thread slot s (mixed-width heads: rows
+                              //         grouped by width, so a warp's rows share a width); else s
   const float* col;           // [h_v*d] c_j
   const float* icol;          // [h_v*d] fl(1 / c_j)
   const float* phi;           // [h_v*d] phi_i
@@ -142,13 +144,13 @@ struct Geo {
   static constexpr int NT = 32 * NW;          // threads per CTA
   static constexpr int NG = NW * RPW;         // row groups (= rows per pass of the CTA)
   static constexpr int RPT = D / NG;          // rows per thread
-  static constexpr int AUX = (31 * D + 32 + 127) / 128 * 128;  // vector bytes per stage (see stage layout)
+  static constexpr int AUX = (32 * D + 32 + 127) / 128 * 128;  // vector bytes per stage (see stage layout)
   static_assert(RPT >= 1 && RPT * NG == D, "bad geometry");
 };
 
 // Stage layout: [k f32 D][q f32 D][v f32 D][g f32 D][c f32 D][ic f32 D]
-//               [phi f32 D][row_off u16 D][row_code u8 D][TileHdr 32 B]
-//               (padded to Geo<D>::AUX bytes) [record: rec_cap]
+//               [phi f32 D][row_off u16 D][row_code u8 D][row_perm u8 D]
+//               [TileHdr 32 B] (padded to Geo<D>::AUX bytes) [record: rec_cap]
 // Every offset but the stage's own base is a compile-time constant.
 template <int D>
 struct Stage {
@@ -163,7 +165,8 @@ struct Stage {
   __device__ float* phi() const { return k() + 6 * D; }
   __device__ uint16_t* row_off() const { return reinterpret_cast<uint16_t*>(k() + 7 * D); }
   __device__ uint8_t* row_code() const { return reinterpret_cast<uint8_t*>(row_off() + D); }
-  __device__ struct TileHdr* hdr() const { return reinterpret_cast<struct TileHdr*>(row_code() + D); }
+  __device__ uint8_t* row_perm() const { return row_code() + D; }
+  __device__ struct TileHdr* hdr() const { return reinterpret_cast<struct TileHdr*>(row_perm() + D); }
   __device__ uint8_t* rec() const { return base + Geo<D>::AUX; }
 };
 
@@ -300,11 +303,13 @@ template <int B, int H>
 __device__ __forceinline__ void hi_half_q(const uint32_t (&w)[B / 2], uint32_t (&xh)[8], float2 (&V)[4]) {
 #pragma unroll
   for (int j = 0; j < 8; ++j) xh[j] = field_hi<B>(w, 8 * H + j);
+  // scalar fmas: each value lands directly in its pair register (an f32x2
+  // fma would need xh[2p], xh[2p+1] in an aligned pair, which the fp64 views
+  // of the same words also claim)
   constexpr float K = FieldPos<B>::K, C = FieldPos<B>::C;
 #pragma unroll
   for (int p = 0; p < 4; ++p)
-    V[p] = __ffma2_rn(make_float2(__uint_as_float(xh[2 * p]), __uint_as_float(xh[2 * p + 1])), make_float2(K, K),
-                      make_float2(-C, -C));
+    V[p] = make_float2(__fmaf_rn(__uint_as_float(xh[2 * p]), K, -C), __fmaf_rn(__uint_as_float(xh[2 * p + 1]), K, -C));
 }
 // Pivot chunk: the fp16 values themselves (an fp16 value as a double has a
 // zero low word).
@@ -608,16 +613,14 @@ __device__ __forceinline__ float column_sum(float* red, int rg, int cc, const fl
 }
 
 // fp64 deposit of the 8 partials of half `half` of a thread's 16 columns
-// (same swizzle idea: 16-byte chunks of two doubles rotated by cc), minus
-// the thread's per-row offsets.
+// (same swizzle idea: 16-byte chunks of two doubles rotated by cc).
 template <int D>
-__device__ __forceinline__ void deposit_f64(double* red, int rg, int cc, int half, const double (&acc)[8],
-                                            double off) {
+__device__ __forceinline__ void deposit_f64(double* red, int rg, int cc, int half, const double (&acc)[8]) {
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const int chunk = 4 * half + p;
     *reinterpret_cast<double2*>(red + rg * D + 16 * cc + 2 * (chunk ^ (cc & 7))) =
-        make_double2(acc[2 * p] - off, acc[2 * p + 1] - off);
+        make_double2(acc[2 * p], acc[2 * p + 1]);
   }
 }
 
@@ -969,7 +972,8 @@ __device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalar
   hd->beta = x.beta;
   hd->g = x.g;
   hd->kind = x.kind;
-  uint32_t tx = 6u * vec + (kda ? vec : 0u) + 3u * D;
+  const bool mixed = x.kind == 0;  // rows of different widths: the row order is needed
+  uint32_t tx = 6u * vec + (kda ? vec : 0u) + 3u * D + (mixed ? (uint32_t)D : 0u);
   if (!direct) tx += x.rec_bytes;
   mbar_arrive_expect_tx(bar, tx);
   if (direct)
@@ -985,6 +989,7 @@ __device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalar
   bulk_g2s(s.phi(), a.t.phi + (size_t)h * D, vec, bar);
   bulk_g2s(s.row_off(), a.t.row_off + (size_t)h * D, 2u * D, bar);
   bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
+  if (mixed) bulk_g2s(s.row_perm(), a.t.row_perm + (size_t)h * D, (uint32_t)D, bar);
 }
 
 // Thread 0: issue the next tile into stage s (or mark the stage as the end
@@ -1049,13 +1054,13 @@ __device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, 
 // acc. Only the words of half H are loaded.
 template <int D, int B, int H, bool DIRECT>
 __device__ __forceinline__ void pass_a_half(const uint8_t* rec, int rg, int cc, const double (&kap)[Geo<D>::RPT],
-                                            float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
+                                            double acc0, float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
   uint32_t w[Geo<D>::RPT][B / 2];
 #pragma unroll
   for (int r = 0; r < Geo<D>::RPT; ++r)
     chunk_words<B, DIRECT>(rec + row_offset<D, B>(nullptr, r * Geo<D>::NG + rg), cc, w[r]);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+  for (int j = 0; j < 8; ++j) acc[j] = acc0;
 #pragma unroll
   for (int r = 0; r < Geo<D>::RPT; ++r) {
     uint32_t xh[8];
@@ -1079,14 +1084,15 @@ __device__ __forceinline__ void pass_a_half(const uint8_t* rec, int rg, int cc, 
 // gave up).
 template <int D, int H>
 __device__ __forceinline__ void pass_a_half_mixed(const uint8_t* rec, const uint16_t* row_off,
-                                                  const uint8_t* row_code, uint32_t rec_cap, int rg, int cc,
-                                                  const double (&kap)[Geo<D>::RPT], float2 (&T)[Geo<D>::RPT][8],
-                                                  double (&acc)[8]) {
+                                                  const uint8_t* row_code, const uint8_t* row_perm,
+                                                  uint32_t rec_cap, int rg, int cc,
+                                                  const double (&kap)[Geo<D>::RPT], double acc0,
+                                                  float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+  for (int j = 0; j < 8; ++j) acc[j] = acc0;
 #pragma unroll
   for (int r = 0; r < Geo<D>::RPT; ++r) {
-    const int i = r * Geo<D>::NG + rg;
+    const int i = row_perm[r * Geo<D>::NG + rg] & (D - 1);  // (masked: in bounds even if never loaded)
     const uint8_t* row = rec + min((uint32_t)row_off[i], rec_cap);
     uint32_t xh[8];
     float2 V[4];
@@ -1137,8 +1143,8 @@ __device__ __forceinline__ float row_absmax(const float2 (&t)[8]) {
 // per-row tests.
 template <int D, int KC, int RB>
 __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
-                                                  const float* phi, int grp, int rg, int cc,
-                                                  const float2 (&T)[RB][8]) {
+                                                  const uint8_t* row_perm, const float* phi, int grp, int rg,
+                                                  int cc, const float2 (&T)[RB][8]) {
   using G = Geo<D>;
   uint32_t st = 0;
   if constexpr (KC == ROW_PIVOT) {
@@ -1158,7 +1164,8 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
     float mm = m[0];
 #pragma unroll
     for (int u = 1; u < RB; ++u) mm = mine == u ? m[u] : mm;
-    const int im = (grp * RB + mine) * G::NG + rg;
+    const int sm = (grp * RB + mine) * G::NG + rg;  // slot
+    const int im = KC ? sm : row_perm[sm];           // row
     const int cm = KC ? KC : row_code[im];
     float ir_m = 0.0f;
     if (cm != ROW_PIVOT) {
@@ -1184,7 +1191,7 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
-        const int i = (grp * RB + u) * G::NG + rg;
+        const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
         const int code = KC ? KC : row_code[i];
         uint8_t* row = rec + row_offset<D, KC>(row_off, i);
         switch (code) {
@@ -1199,7 +1206,7 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
-        const int i = (grp * RB + u) * G::NG + rg;
+        const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
         const int code = KC ? KC : row_code[i];
         uint8_t* row = rec + row_offset<D, KC>(row_off, i);
         if (code == ROW_PIVOT) {
@@ -1251,36 +1258,40 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
     // by shuffle. M = fp32(r g) (quantized row) or g (pivot row); the fp64
     // weight kap = M k is exact.
     const int mine = cc % G::RPT;
-    const int im = mine * G::NG + rg;
+    const int sm = mine * G::NG + rg;                  // slot
+    const int im = KC ? sm : (S.row_perm()[sm] & (D - 1));  // row (masked: in bounds even if never loaded)
     const int cm = KC ? KC : S.row_code()[im];
     const float gm = kda ? S.g()[im] : hd->g;
     const float mm =
         cm == ROW_PIVOT ? gm : __fmul_rn(__half2float(reinterpret_cast<const __half*>(rec)[im]), gm);
-    if (cc < G::RPT) msh[im] = mm;
+    if (cc < G::RPT) msh[sm] = mm;
     const double kapm = (double)mm * (double)S.k()[im];
     double kap[G::RPT];
     double off = 0.0;
 #pragma unroll
     for (int r = 0; r < G::RPT; ++r) {
       kap[r] = __shfl_sync(0xffffffffu, kapm, base + r);
-      const int code = KC ? KC : S.row_code()[r * G::NG + rg];
+      const int code = KC ? KC : S.row_code()[S.row_perm()[r * G::NG + rg] & (D - 1)];
       if (code != ROW_PIVOT) off = fma(code_offset(code), kap[r], off);
     }
     bool free_ok = true;
     double acc[8];
+    // the accumulators start at -off, the rows' bias (see code_offset)
     if constexpr (KC != 0) {
-      pass_a_half<D, KC, 0, DIRECT>(rec, rg, cc, kap, T, acc);
+      pass_a_half<D, KC, 0, DIRECT>(rec, rg, cc, kap, -off, T, acc);
       // the buffer is free once every thread has read the previous tile's o partials
       if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc, off);
-      pass_a_half<D, KC, 1, DIRECT>(rec, rg, cc, kap, T, acc);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc, off);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc);
+      pass_a_half<D, KC, 1, DIRECT>(rec, rg, cc, kap, -off, T, acc);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc);
     } else {
-      pass_a_half_mixed<D, 0>(rec, S.row_off(), S.row_code(), a.rec_cap, rg, cc, kap, T, acc);
+      pass_a_half_mixed<D, 0>(rec, S.row_off(), S.row_code(), S.row_perm(), a.rec_cap, rg, cc, kap, -off, T,
+                              acc);
       if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc, off);
-      pass_a_half_mixed<D, 1>(rec, S.row_off(), S.row_code(), a.rec_cap, rg, cc, kap, T, acc);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc, off);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc);
+      pass_a_half_mixed<D, 1>(rec, S.row_off(), S.row_code(), S.row_perm(), a.rec_cap, rg, cc, kap, -off, T,
+                              acc);
+      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc);
     }
     if (!free_ok) *abort_sh = 1;
   }
@@ -1314,15 +1325,16 @@ __device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S
   float2 part[8];
 #pragma unroll
   for (int r = 0; r < G::RPT; ++r) {
-    const int i = r * G::NG + rg;
-    const float kr = S.k()[i], qr = S.q()[i], M = msh[i];
+    const int sl = r * G::NG + rg;
+    const int i = KC ? sl : S.row_perm()[sl];
+    const float kr = S.k()[i], qr = S.q()[i], M = msh[sl];
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       T[r][p] = __ffma2_rn(T[r][p], f2(M), __fmul2_rn(f2(kr), W[p]));
       part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr)) : __ffma2_rn(T[r][p], f2(qr), part[p]);
     }
   }
-  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.phi(), 0, rg, cc, T);
+  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.row_perm(), S.phi(), 0, rg, cc, T);
   column_deposit<D>(reinterpret_cast<float*>(red), rg, cc, part);
   if (!DIRECT) fence_proxy_async_smem();  // the new record is read by the bulk store
   __syncthreads();  // B3: the o partials and the new record are complete

@@ -41,7 +41,7 @@ def main():
         for t in range(2):
             q, k, v, beta, g = w.step_inputs(t)
             o = np.zeros((c.batch, c.h_v, c.d), dtype=np.float32)
-            o_.step(pool, q, k, v, beta, g, o)
+            o_.step(pool, q, k, v, beta, g, o=o)
             outs.append(o)
         dist.barrier()
         mx = shards.max_over_ranks(float(10 * (rank + 1)), dist)

@@ -43,7 +43,7 @@ def _single_process(seed):
     for t in range(2):
         q, k, v, beta, g = w.step_inputs(t)
         o = np.zeros((c.batch, c.h_v, c.d), dtype=np.float32)
-        o_.step(pool, q, k, v, beta, g, o)
+        o_.step(pool, q, k, v, beta, g, o=o)
         outs.append(o)
     return np.stack(outs), pool
 
@@ -72,6 +72,7 @@ def test_two_ranks_shard_requests_with_no_data_collective(tmp_path):
     # ... and its result is exactly that of a single process on the same shard
     for r in range(world):
         o_ref, pool_ref = _single_process(shards.rank_seed(11, r))
+        assert np.abs(o_ref).max() > 0
         np.testing.assert_array_equal(res[r]["o"], o_ref)
         np.testing.assert_array_equal(res[r]["pool"], pool_ref)
     # measurement collectives: the slowest rank's time, the whole-job rate
