@@ -45,6 +45,28 @@ def trace_moments(states: np.ndarray) -> np.ndarray:
     return m2
 
 
+def token_mean_square(x: np.ndarray) -> np.ndarray:
+    """E[x^2] over the leading (token) axis: the sum over tokens, in order,
+    of x^2 in fp64, divided by the token count (fp64). Used for the queries'
+    second moments [h_k, d]."""
+    x = np.asarray(x, dtype=np.float32)
+    acc = np.zeros(x.shape[1:], dtype=np.float64)
+    for t in range(x.shape[0]):
+        v = x[t].astype(np.float64)
+        acc += v * v
+    return acc / x.shape[0]
+
+
+def token_mean(x: np.ndarray) -> np.ndarray:
+    """Mean over the leading (token) axis: the sum over tokens, in order, in
+    fp64, divided by the token count. Used for each unit's mean gate."""
+    x = np.asarray(x, dtype=np.float32)
+    acc = np.zeros(x.shape[1:], dtype=np.float64)
+    for t in range(x.shape[0]):
+        acc += x[t].astype(np.float64)
+    return acc / x.shape[0]
+
+
 def _geomean_normalised(x: np.ndarray) -> np.ndarray:
     """x / geomean(x) over the last axis, x > 0 (fp64)."""
     lg = np.log(x)
@@ -165,6 +187,16 @@ def allocate(sigma2: np.ndarray, weight: np.ndarray, widths, nominal: int, pivot
         budget -= nxt[int(bits[best])] - int(bits[best])
         bits[best] = nxt[int(bits[best])]
     return bits.astype(np.int8), pivot
+
+
+def calibrate_from_trace(states, q_tokens, g_tokens, per_row: bool, widths, nominal: int,
+                         pivot_frac: float):
+    """Calibration from raw traces: states [n, h_v, d, d] (fp32 S samples),
+    q_tokens [n_q, h_k, d] and g_tokens [n_g, h_v] (per head) or
+    [n_g, h_v, d] (per key channel). A unit's retention is its mean gate over
+    the tokens; a row's raw impact is the queries' mean square."""
+    return calibrate(states, token_mean_square(q_tokens), token_mean(g_tokens), per_row, widths, nominal,
+                     pivot_frac)
 
 
 def calibrate(states, q_sq, gates, per_row: bool, widths, nominal: int, pivot_frac: float):

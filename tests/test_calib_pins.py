@@ -148,3 +148,42 @@ def test_calibrate_end_to_end_shapes_and_invariants():
     assert int(bits.sum()) <= 6 * h_v * d
     assert np.all(c > 0) and np.all(np.isfinite(c))
     assert np.allclose(np.exp(np.log(phi.astype(np.float64)).mean(axis=1)), 1.0, rtol=1e-6)
+
+
+def test_trace_moments_exact_on_integers():
+    # small integers: every square and partial sum is exact in fp64, so the
+    # result equals exact integer arithmetic
+    rng = np.random.default_rng(11)
+    states = rng.integers(-2000, 2001, size=(9, 2, 4, 4))
+    m2 = oc.trace_moments(states.astype(np.float32))
+    want = (states.astype(object) ** 2).sum(axis=0)
+    assert np.array_equal(m2.astype(np.int64), want.astype(np.int64))
+
+
+def test_trace_moments_order_is_sequential():
+    # 1 followed by many values whose squares are below half an ulp of the
+    # running sum: a sequential fp64 sum never moves, a pairwise one would
+    tiny = np.float32(2.0 ** -27)          # tiny^2 = 2^-54 = half an ulp of 1.0
+    states = np.full((64, 1, 1, 1), tiny, np.float32)
+    states[0] = 1.0
+    assert oc.trace_moments(states)[0, 0, 0] == 1.0
+
+
+def test_token_means_closed_form():
+    q = np.broadcast_to(np.array([0.5, -2.0, 3.0], np.float32), (7, 1, 3))
+    assert np.array_equal(oc.token_mean_square(q), [[0.25, 4.0, 9.0]])
+    g = np.array([[0.5], [0.75], [1.0], [0.25]], np.float32)
+    assert np.array_equal(oc.token_mean(g), [0.625])
+
+
+def test_calibrate_from_trace_constant_tokens_matches_direct():
+    rng = np.random.default_rng(5)
+    h_v, h_k, d = 2, 1, 8
+    states = rng.normal(0, 1, size=(4, h_v, d, d)).astype(np.float32)
+    qrow = rng.uniform(0.5, 2, size=(h_k, d)).astype(np.float32)
+    grow = np.array([0.5, 0.875], np.float32)
+    a = oc.calibrate_from_trace(states, np.broadcast_to(qrow, (5, h_k, d)), np.broadcast_to(grow, (3, h_v)),
+                                False, (4, 6, 8), 6, 0.0)
+    b = oc.calibrate(states, qrow.astype(np.float64) ** 2, grow, False, (4, 6, 8), 6, 0.0)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
