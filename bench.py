@@ -469,15 +469,84 @@ def run_rollout(args, rank, world, local_rank):
         print(json.dumps(out), flush=True)
 
 
+def run_calibration(args, rank, world, local_rank):
+    """The calibration workload on the serving layer's shape (32 value heads,
+    16 key heads, d = 128, GDN): a 512-sample fp32 state trace (1 GiB, beyond
+    L2) and 4096 tokens of queries and gates (synthetic, seeded). The timed
+    kernel is the trace pass (fp64 running sums of S^2, one launch per pass
+    over the whole trace); the whole calibration (accumulators, trace pass,
+    token pass, tables, allocation) is timed on the host clock around a
+    synchronised run. Prints its own JSON line."""
+    import torch
+    from quantized_linear_attention_sq_b200 import build, shards, synth
+    from quantized_linear_attention_sq_b200.calibrate import TraceCalibrator
+
+    torch.cuda.set_device(local_rank)
+    build.build()
+    dev = torch.device("cuda", local_rank)
+    c = synth.CONFIGS[CONFIG_ID]
+    n_states, n_tok = args.trace_samples, 4096
+    states, q, g = synth.calibration_trace(c.h_v, c.h_k, c.d, c.gate_kind, n_states, n_tok,
+                                           seed=shards.rank_seed(args.seed, rank))
+    S = torch.from_numpy(states).to(dev)
+    qd, gd = torch.from_numpy(q).to(dev), torch.from_numpy(g).to(dev)
+    del states
+    stream = torch.cuda.current_stream()
+    cal = TraceCalibrator(c.h_v, c.h_k, c.d, c.gate_kind)
+    for _ in range(args.warmup):
+        cal.add_states(S)
+    torch.cuda.synchronize()
+    K = max(1, min(args.steps, 200))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            cal.add_states(S)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    cal.close()
+    # the whole calibration, once more from empty accumulators
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    cal = TraceCalibrator(c.h_v, c.h_k, c.d, c.gate_kind)
+    cal.add_states(S)
+    cal.add_tokens(qd, gd)
+    tabs = cal.finish(c.widths, c.nominal_bits, c.pivot_frac)
+    whole_ms = (time.perf_counter() - t0) * 1e3
+    cal.close()
+    E = c.h_v * c.d * c.d
+    alg_bytes = n_states * E * 4 + 2 * E * 8
+    peak, peak_kind = peaks()
+    achieved = alg_bytes / (ms / 1e3) / 1e9
+    out = {"metric": "calibration trace pass, state samples/s", "unit": "state-samples/s", "n_gpus": world,
+           "steps": K, "warmup": args.warmup, "ms_per_step": ms, "value": n_states * c.h_v / (ms / 1e3),
+           "higher_is_better": True, "dtype": "f64 sums of f32", "data": "synthetic",
+           "config": {"workload": "calib_trace_gdn_hv32_hk16_d128", "trace_samples": n_states,
+                      "tokens": n_tok, "trace_bytes": n_states * E * 4, "l2": f"{n_states * E * 4 / 2**20:.0f} MiB trace > 126 MB L2"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "kernel": "k_trace_sum<4,true>",
+                        "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+           "whole_calibration_ms": whole_ms,
+           "tables": {"pivot_heads": int(tabs.pivot.sum()),
+                      "widths": {str(b): int((tabs.unit_bits[tabs.pivot == 0] == b).sum()) for b in c.widths}},
+           "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers"], default="serving",
+    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers", "calibration"], default="serving",
                     help="serving: the headline GDN workload; kda_rollout_8layers: 8 KDA layers, "
-                         "per-layer launches vs one CUDA graph")
+                         "per-layer launches vs one CUDA graph; calibration: the trace pass of the "
+                         "calibration library on the serving layer's shape")
+    ap.add_argument("--trace-samples", type=int, default=512,
+                    help="calibration workload: state samples in the trace (512 = 1 GiB)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -494,6 +563,8 @@ def main():
         run_reference(args, rank, world)
     elif args.workload == "kda_rollout_8layers":
         run_rollout(args, rank, world, local_rank)
+    elif args.workload == "calibration":
+        run_calibration(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

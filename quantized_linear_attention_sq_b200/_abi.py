@@ -7,6 +7,7 @@ cannot be loaded, ``lib()`` raises.
 from __future__ import annotations
 
 import ctypes
+import glob
 import os
 import re
 
@@ -56,6 +57,16 @@ class BytesReport(ctypes.Structure):
                 ("bits_per_value", ctypes.c_double), ("max_record_bytes", ctypes.c_uint64)]
 
 
+class CalibBudget(ctypes.Structure):
+    _fields_ = [("widths_mask", ctypes.c_int32), ("nominal_bits", ctypes.c_int32), ("pivot_frac", ctypes.c_double)]
+
+
+class CalibOut(ctypes.Structure):
+    _fields_ = [("unit_bits", ctypes.c_void_p), ("pivot_mask", ctypes.c_void_p), ("col_scale", ctypes.c_void_p),
+                ("row_impact", ctypes.c_void_p), ("unit_sigma2", ctypes.c_void_p),
+                ("unit_weight", ctypes.c_void_p)]
+
+
 _lib = None
 
 
@@ -86,18 +97,27 @@ def lib() -> ctypes.CDLL:
     L.sq_version.restype = ctypes.c_char_p
     L.sq_decode_step_noalloc.argtypes = [ctypes.POINTER(StateDesc), ctypes.POINTER(Calib)] + [P] * 8 + [I32, P, P]
     L.sq_decode_step_noalloc.restype = ctypes.c_int
+    L.sq_calib_begin.argtypes = [ctypes.POINTER(StateDesc), P, ctypes.POINTER(P)]
+    L.sq_calib_add_states.argtypes = [P, P, I32, P]
+    L.sq_calib_add_tokens.argtypes = [P, P, P, I32, P]
+    L.sq_calib_finish.argtypes = [P, ctypes.POINTER(CalibBudget), ctypes.POINTER(CalibOut), P]
+    L.sq_calib_free.argtypes = [P]
     for name in ("sq_state_alloc", "sq_state_free", "sq_quantize_state", "sq_decode_step",
-                 "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status"):
+                 "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status",
+                 "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
+                 "sq_calib_free"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
 
 
 def header_functions() -> list:
-    """Names of the functions include/sq.h declares."""
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(sq_[a-z_]+)\s*\(", text)))
+    """Names of the functions the headers under include/ declare."""
+    names = set()
+    for path in sorted(glob.glob(os.path.join(os.path.dirname(HEADER), "*.h"))):
+        text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names.update(re.findall(r"\b(sq_[a-z_]+)\s*\(", text))
+    return sorted(names)
 
 
 def check(code: int) -> None:
@@ -160,3 +180,25 @@ def sq_decode_step_noalloc(desc: StateDesc, calib: Calib, pool, q, k, v, beta, g
 
 def sq_version() -> str:
     return lib().sq_version().decode()
+
+
+def sq_calib_begin(desc: StateDesc, stream: int):
+    t = ctypes.c_void_p()
+    check(lib().sq_calib_begin(ctypes.byref(desc), ctypes.c_void_p(stream), ctypes.byref(t)))
+    return t
+
+
+def sq_calib_add_states(t, S: int, n: int, stream: int) -> None:
+    check(lib().sq_calib_add_states(t, S, n, stream))
+
+
+def sq_calib_add_tokens(t, q: int | None, g: int | None, n: int, stream: int) -> None:
+    check(lib().sq_calib_add_tokens(t, q, g, n, stream))
+
+
+def sq_calib_finish(t, budget: CalibBudget, out: CalibOut, stream: int) -> None:
+    check(lib().sq_calib_finish(t, ctypes.byref(budget), ctypes.byref(out), stream))
+
+
+def sq_calib_free(t) -> None:
+    check(lib().sq_calib_free(t))

@@ -11,9 +11,10 @@
 #include <vector>
 
 #include "sq.h"
+#include "sq_host.h"
 #include "sq_kernels.cuh"
 
-namespace {
+namespace sqi {
 
 thread_local std::string g_last_error;
 
@@ -30,6 +31,14 @@ sq_status fail(sq_status s, const char* fmt, ...) {
 sq_status cuda_fail(cudaError_t e, const char* what) {
   return fail(SQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
+
+}  // namespace sqi
+
+using sqi::cuda_fail;
+using sqi::fail;
+using sqi::g_last_error;
+
+namespace {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

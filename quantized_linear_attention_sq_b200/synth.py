@@ -35,6 +35,7 @@ GATE_KEY_CHANNEL = 1   # KDA: one gate per key channel
 _STREAM_CALIB = 0
 _STREAM_STATE = 1
 _STREAM_STEP = 2
+_STREAM_TRACE = 3
 
 
 @dataclass(frozen=True)
@@ -216,3 +217,36 @@ class Workload:
 
 def workload(cid: int, seed: int = 0, layer: int = 0, batch: int | None = None) -> Workload:
     return Workload(CONFIGS[cid], seed=seed, layer=layer, batch=batch)
+
+
+def calibration_trace(h_v: int, h_k: int, d: int, gate_kind: int, n_states: int, n_tokens: int, seed: int = 0,
+                      col_sigma: float = 0.5, row_sigma: float = 0.5, q_sigma: float = 0.5,
+                      half_life_max: float = 4096.0, outlier_frac: float = 0.02, outlier_gain: float = 20.0,
+                      state_std: float = 0.1):
+    """A seeded synthetic calibration trace of one layer.
+
+    states [n_states, h_v, d, d] fp32: N(0, state_std) times a per-(head, key
+    row) magnitude lognormal(0, row_sigma) times a per-(head, value column)
+    magnitude lognormal(0, col_sigma), with outlier_gain on outlier_frac of
+    each head's columns; q [n_tokens, h_k, d] fp32: N(0, 1) times a
+    per-channel RMS lognormal(0, q_sigma); g [n_tokens, h_v] (per head) or
+    [n_tokens, h_v, d] (per key channel) fp32: each unit's base retention
+    2^(-1/h) with h log-uniform in [1, half_life_max], raised per token to a
+    power lognormal(0, 0.2) (so every gate stays in (0, 1)).
+    """
+    rng = _rng(seed, h_v, h_k, d, gate_kind, _STREAM_TRACE)
+    row = np.exp(rng.normal(0.0, row_sigma, size=(h_v, d, 1)))
+    col = np.exp(rng.normal(0.0, col_sigma, size=(h_v, 1, d)))
+    n_out = round_half_up(outlier_frac * d)
+    for h in range(h_v):
+        col[h, 0, rng.choice(d, size=n_out, replace=False)] *= outlier_gain
+    mag = (state_std * row * col).astype(np.float32)
+    states = np.empty((n_states, h_v, d, d), dtype=np.float32)
+    for t in range(n_states):
+        states[t] = rng.standard_normal(size=(h_v, d, d), dtype=np.float32) * mag
+    q = (rng.standard_normal(size=(n_tokens, h_k, d)) *
+         np.exp(rng.normal(0.0, q_sigma, size=(h_k, d)))).astype(np.float32)
+    shape = (h_v,) if gate_kind == GATE_HEAD else (h_v, d)
+    base = np.power(2.0, -1.0 / np.exp(rng.uniform(0.0, np.log(half_life_max), size=shape)))
+    g = np.power(base, np.exp(rng.normal(0.0, 0.2, size=(n_tokens,) + shape))).astype(np.float32)
+    return states, q, g

@@ -108,3 +108,24 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(ImportError):
         _abi.lib()
+
+
+@pytest.mark.parametrize("kw,code,needle", [
+    (dict(d_k=48, d_v=48), _abi.SQ_ERR_UNSUPPORTED, "d must be"),
+    (dict(h_v=6, h_k=4), _abi.SQ_ERR_INVALID_ARG, "multiple"),
+    (dict(h_k=0), _abi.SQ_ERR_INVALID_ARG, "positive"),
+    (dict(gate=2), _abi.SQ_ERR_INVALID_ARG, "gate"),
+])
+def test_calib_begin_rejects_bad_descriptions(L, kw, code, needle):
+    t = ctypes.c_void_p()
+    rc = L.sq_calib_begin(ctypes.byref(_desc(**kw)), None, ctypes.byref(t))
+    assert rc == code and needle in L.sq_last_error().decode() and not t.value
+
+
+def test_calib_calls_reject_null_arguments(L):
+    assert L.sq_calib_add_states(None, None, 1, None) == _abi.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_add_tokens(None, None, None, 1, None) == _abi.SQ_ERR_INVALID_ARG
+    budget = _abi.CalibBudget(1 << 6, 6, 0.0)
+    out = _abi.CalibOut()
+    assert L.sq_calib_finish(None, ctypes.byref(budget), ctypes.byref(out), None) == _abi.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_free(None) == _abi.SQ_OK
