@@ -535,18 +535,78 @@ def run_calibration(args, rank, world, local_rank):
         print(json.dumps(out), flush=True)
 
 
+def run_prefill(args, rank, world, local_rank):
+    """The prefill handoff on the serving shape (512 requests x 32 value
+    heads, 16 key heads, d = 128, GDN, the serving calibration): a prompt of
+    --prompt-len tokens per request from a zero state, every (request, head)
+    state kept on chip over the prompt and quantized once into its pool slot.
+    One launch per step. Bound by fp32 arithmetic: 7 d^2 flops per (request,
+    head, token) (gate d^2, S^T k 2d^2, update 2d^2, S^T q 2d^2). Prints its
+    own JSON line."""
+    import torch
+    from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
+    from quantized_linear_attention_sq_b200.state import StatePool
+
+    torch.cuda.set_device(local_rank)
+    build.build()
+    dev = torch.device("cuda", local_rank)
+    w = synth.workload(CONFIG_ID, seed=shards.rank_seed(args.seed, rank))
+    c = w.cfg
+    B, L = c.batch, args.prompt_len
+    cal = w.calib()
+    sp = StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, _abi.SQ_FMT_PACKED, cal.unit_bits, cal.pivot,
+                   cal.col_scale, cal.row_impact)
+    pool = sp.new_pool()
+    prompt = [torch.from_numpy(x).to(dev) for x in w.prompt_inputs(L)]
+    o = torch.empty((B, L, c.h_v, c.d), device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        sp.prefill(pool, *prompt, o)
+    torch.cuda.synchronize()
+    K = max(1, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(K):
+            sp.prefill(pool, *prompt, o)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    status = sp.get_status()
+    sp.close()
+    clocks = clk.summary()
+    flops = 7.0 * c.d * c.d * B * c.h_v * L
+    sm_mhz = clocks.get("sm_max_mhz") or 1965.0
+    peak_tflops = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    achieved = flops / (ms / 1e3) / 1e12
+    out = {"metric": "prefill handoff, prompt tokens/s", "unit": "request-tokens/s", "n_gpus": world,
+           "steps": K, "warmup": args.warmup, "ms_per_step": ms, "value": B * L * world / (ms / 1e3),
+           "higher_is_better": True, "scaling": "weak", "dtype": "f32", "data": "synthetic",
+           "config": {"workload": f"prefill_gdn_b{B}_hv{c.h_v}_hk{c.h_k}_d{c.d}_L{L}", "batch_per_gpu": B,
+                      "prompt_len": L, "handoff": "quantized once into the packed pool (6-bit nominal)"},
+           "roofline": {"bound": "alu", "achieved": achieved, "peak": peak_tflops, "unit": "TFLOP/s",
+                        "frac": achieved / peak_tflops, "kernel": "k_prefill<128>",
+                        "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock"},
+           "status_bits": status, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers", "calibration"], default="serving",
+    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers", "calibration", "prefill"],
+                    default="serving",
                     help="serving: the headline GDN workload; kda_rollout_8layers: 8 KDA layers, "
                          "per-layer launches vs one CUDA graph; calibration: the trace pass of the "
-                         "calibration library on the serving layer's shape")
+                         "calibration library on the serving layer's shape; prefill: the prefill "
+                         "handoff on the serving shape")
     ap.add_argument("--trace-samples", type=int, default=512,
                     help="calibration workload: state samples in the trace (512 = 1 GiB)")
+    ap.add_argument("--prompt-len", type=int, default=128, help="prefill workload: tokens per prompt")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -565,6 +625,8 @@ def main():
         run_rollout(args, rank, world, local_rank)
     elif args.workload == "calibration":
         run_calibration(args, rank, world, local_rank)
+    elif args.workload == "prefill":
+        run_prefill(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank)
 

@@ -154,6 +154,34 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
 sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, const int32_t* slot_ids,
                               int32_t B, void* stream);
 
+/* Prefill handoff: run the gated delta rule over a whole prompt for B
+ * requests and write the final state once into their pool slots, quantized
+ * for SQ_FMT_PACKED ("STEPQuant review (e-cogni)", "Contexto": the state a
+ * prompt leaves behind is what every decode step then updates; "O que os
+ * autores propõem": it enters the cache in the dual-axis quantized form).
+ * One launch; each (request, head) state stays on chip for the whole
+ * prompt. Token t of request b applies exactly the FP32 decode step of
+ * sq_decode_step on an SQ_FMT_FP32 pool (same arithmetic and summation
+ * order), so the final fp32 state equals that of L such steps bit for bit;
+ * the quantization is that of sq_quantize_state.
+ *   S0       device fp32 [B, h_v, d, d] initial state, or NULL for zeros
+ *   q, k     device fp32 [B, L, h_k, d]
+ *   v        device fp32 [B, L, h_v, d]
+ *   beta     device fp32 [B, L, h_v]
+ *   g        device fp32 [B, L, h_v] (GATE_HEAD) or [B, L, h_v, d] (GATE_KEY_CHANNEL)
+ *   o        device fp32 [B, L, h_v, d], written for t < lengths[b]: o_t = S_t^T q_t
+ *   S_out    device fp32 [B, h_v, d, d] final state (unquantized), or NULL
+ *   lengths  device int32 [B] prompt lengths (values outside [0, L] are
+ *            clamped), or NULL for L; a length of 0 stores S0 (or zeros)
+ *   slot_ids device int32 [B] (distinct), or NULL for slots 0..B-1; an
+ *            out-of-range slot is skipped (SQ_STATUS_BAD_SLOT), o and S_out
+ *            are still written
+ * q, k, v, o, S0 and S_out 16-byte aligned; g too for GATE_KEY_CHANNEL.
+ * B == 0 is a no-op; L == 0 stores S0 (or zeros). */
+sq_status sq_prefill(sq_handle* h, void* pool, const float* S0, const float* q, const float* k, const float* v,
+                     const float* beta, const float* g, float* o, float* S_out, const int32_t* lengths,
+                     const int32_t* slot_ids, int32_t B, int32_t L, void* stream);
+
 /* Byte accounting of the layout (host only, no device work). */
 sq_status sq_state_bytes(const sq_handle* h, sq_bytes_report* out);
 

@@ -167,6 +167,39 @@ class Oracle:
         assert S.dtype == np.float32 and S.flags.c_contiguous
         return self._run_tiles(lib().sqo_step_fp32_tiles, S, q, k, v, beta, g, slots, o, threads, tiles)
 
+    def prefill(self, pool, S0, q, k, v, beta, g, lengths=None, slots=None, fp32_pool=False):
+        """Prefill handoff: the gated delta rule token by token over each
+        prompt (the unquantized step above, in token order), then the final
+        state written once into the request's slot: quantized (``pool``
+        packed) or as fp32 (``fp32_pool``: ``pool`` is [n_slots, h_v, d, d]).
+        q, k [B, L, h_k, d]; v [B, L, h_v, d]; beta [B, L, h_v]; g [B, L, h_v]
+        or [B, L, h_v, d]; S0 [B, h_v, d, d] or None (zeros); lengths [B]
+        (clamped to [0, L]) or None. Returns (o [B, L, h_v, d], zero past a
+        prompt's end; the final fp32 states [B, h_v, d, d]; status)."""
+        B, L = q.shape[0], q.shape[1]
+        o = np.zeros((B, L, self.h_v, self.d), dtype=np.float32)
+        S_fin = np.zeros((B, self.h_v, self.d, self.d), dtype=np.float32)
+        st = 0
+        for b in range(B):
+            n = L if lengths is None else min(max(int(lengths[b]), 0), L)
+            S = np.zeros((1, self.h_v, self.d, self.d), dtype=np.float32) if S0 is None else \
+                np.array(S0[b:b + 1], dtype=np.float32, order="C")
+            for t in range(n):
+                ob, s = self.step_fp32(S, q[b:b + 1, t], k[b:b + 1, t], v[b:b + 1, t], beta[b:b + 1, t],
+                                       g[b:b + 1, t])
+                o[b, t] = ob[0]
+                st |= s
+            S_fin[b] = S[0]
+            slot = b if slots is None else int(slots[b])
+            if 0 <= slot < self.n_slots:
+                if fp32_pool:
+                    pool[slot] = S[0]
+                else:
+                    st |= self.quantize(pool, S, slots=np.array([slot], dtype=np.int32))
+            else:
+                st |= 4
+        return o, S_fin, st
+
     # ------------------------------------------------ record inspection
     def record(self, pool, slot, h):
         off = slot * self.layout.slot_bytes + self.layout.head_offset[h]

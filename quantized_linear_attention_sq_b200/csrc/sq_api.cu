@@ -13,6 +13,7 @@
 #include "sq.h"
 #include "sq_host.h"
 #include "sq_kernels.cuh"
+#include "sq_prefill.cuh"
 
 namespace sqi {
 
@@ -559,6 +560,59 @@ sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, cons
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching dequantize");
+  h->launches++;
+  return SQ_OK;
+}
+
+sq_status sq_prefill(sq_handle* h, void* pool, const float* S0, const float* q, const float* k, const float* v,
+                     const float* beta, const float* g, float* o, float* S_out, const int32_t* lengths,
+                     const int32_t* slot_ids, int32_t B, int32_t L, void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (B < 0 || L < 0) return fail(SQ_ERR_INVALID_ARG, "B and L must be >= 0 (got %d, %d)", B, L);
+  if (B == 0) return SQ_OK;
+  if ((int64_t)B * h->desc.h_v > (int64_t)INT32_MAX / 2) return fail(SQ_ERR_INVALID_ARG, "B too large");
+  SQ_CHECK_PTR(pool, "pool");
+  if (L > 0) {
+    SQ_CHECK_PTR(q, "q");
+    SQ_CHECK_PTR(k, "k");
+    SQ_CHECK_PTR(v, "v");
+    SQ_CHECK_PTR(o, "o");
+    if (!beta) return fail(SQ_ERR_INVALID_ARG, "beta is NULL");
+    if (!g) return fail(SQ_ERR_INVALID_ARG, "g is NULL");
+    if (h->desc.gate == SQ_GATE_KEY_CHANNEL && !aligned16(g))
+      return fail(SQ_ERR_INVALID_ARG, "g is not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+      return fail(SQ_ERR_INVALID_ARG, "beta/g not 4-byte aligned");
+  }
+  if (S0 && !aligned16(S0)) return fail(SQ_ERR_INVALID_ARG, "S0 is not 16-byte aligned");
+  if (S_out && !aligned16(S_out)) return fail(SQ_ERR_INVALID_ARG, "S_out is not 16-byte aligned");
+  if (lengths && (reinterpret_cast<uintptr_t>(lengths) & 3u)) return fail(SQ_ERR_INVALID_ARG, "lengths misaligned");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  sqk::PrefillArgs a{};
+  a.pool = static_cast<uint8_t*>(pool);
+  a.S0 = S0;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
+  a.S_out = S_out;
+  a.lengths = lengths;
+  a.slots = slot_ids;
+  a.B = B; a.L = L; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots;
+  a.gate_kind = h->desc.gate;
+  a.fmt_fp32 = h->desc.fmt == SQ_FMT_FP32;
+  a.slot_bytes = h->slot_bytes;
+  a.t = h->tables;
+  const int n_tiles = B * h->desc.h_v;
+  const int nt = threads_of(h->d);
+  const uint32_t rec = a.fmt_fp32 ? 0u : (uint32_t)h->max_rec;
+  cudaStream_t st = as_stream(stream);
+  if (h->d == 128)
+    sqk::k_prefill<128><<<n_tiles, nt, sqk::PrefillSmem<128>::bytes(rec), st>>>(a);
+  else if (h->d == 64)
+    sqk::k_prefill<64><<<n_tiles, nt, sqk::PrefillSmem<64>::bytes(rec), st>>>(a);
+  else
+    sqk::k_prefill<32><<<n_tiles, nt, sqk::PrefillSmem<32>::bytes(rec), st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching the prefill");
   h->launches++;
   return SQ_OK;
 }

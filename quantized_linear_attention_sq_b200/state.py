@@ -110,6 +110,22 @@ class StatePool:
                             _ptr(g, torch.float32, "g", gn), _ptr(o, torch.float32, "o", B * hv * d),
                             _ptr(slot_ids, torch.int32, "slot_ids", B), B, _stream(stream))
 
+    def prefill(self, pool, q, k, v, beta, g, o, S0=None, S_out=None, lengths=None, slot_ids=None, stream=None):
+        """Run the prompt (q, k [B, L, h_k, d]; v, o [B, L, h_v, d]; beta [B, L, h_v];
+        g [B, L, h_v] or [B, L, h_v, d]) through the gated delta rule from S0
+        (or zeros) and store the final state once in the requests' slots."""
+        B, L = q.shape[0], q.shape[1]
+        d, hv, hk = self.d, self.h_v, self.h_k
+        gn = B * L * hv * (d if self.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1)
+        n = B * L
+        _abi.sq_prefill(self._h, self._check_pool(pool), _ptr(S0, torch.float32, "S0", B * hv * d * d),
+                        _ptr(q, torch.float32, "q", n * hk * d), _ptr(k, torch.float32, "k", n * hk * d),
+                        _ptr(v, torch.float32, "v", n * hv * d), _ptr(beta, torch.float32, "beta", n * hv),
+                        _ptr(g, torch.float32, "g", gn), _ptr(o, torch.float32, "o", n * hv * d),
+                        _ptr(S_out, torch.float32, "S_out", B * hv * d * d),
+                        _ptr(lengths, torch.int32, "lengths", B), _ptr(slot_ids, torch.int32, "slot_ids", B),
+                        B, L, _stream(stream))
+
     def dequantize_state(self, pool, S_out, slot_ids=None, stream=None):
         B = S_out.shape[0]
         d, hv = self.d, self.h_v

@@ -36,6 +36,7 @@ _STREAM_CALIB = 0
 _STREAM_STATE = 1
 _STREAM_STEP = 2
 _STREAM_TRACE = 3
+_STREAM_PROMPT = 4
 
 
 @dataclass(frozen=True)
@@ -192,6 +193,14 @@ class Workload:
         return m
 
     # ---------------------------------------------------- step inputs
+    def prompt_inputs(self, L: int, requests=None):
+        """A prompt of L tokens per request, drawn token by token like
+        ``step_inputs`` (same distributions, the head's constant gates) from a
+        stream of its own: q, k [n, L, h_k, d], v [n, L, h_v, d], beta
+        [n, L, h_v], g [n, L, h_v] or [n, L, h_v, d]."""
+        toks = [self._token_inputs(_STREAM_PROMPT, t, requests) for t in range(L)]
+        return tuple(np.ascontiguousarray(np.stack([tk[i] for tk in toks], axis=1)) for i in range(5))
+
     def step_inputs(self, step: int, requests=None):
         """Inputs of decode step ``step`` (warm-up steps are -warmup_steps .. -1).
 
@@ -200,8 +209,11 @@ class Workload:
         for requests 0 .. B-1 (or the given request indices). All fp32 and
         C-contiguous.
         """
+        return self._token_inputs(_STREAM_STEP, step, requests)
+
+    def _token_inputs(self, stream: int, step: int, requests):
         c = self.cfg
-        rng = _rng(self.seed, c.cid, self.layer, _STREAM_STEP, step + (1 << 20))
+        rng = _rng(self.seed, c.cid, self.layer, stream, step + (1 << 20))
         B = c.batch
         q = rng.standard_normal(size=(B, c.h_k, c.d))
         k = rng.standard_normal(size=(B, c.h_k, c.d))

@@ -129,3 +129,9 @@ def test_calib_calls_reject_null_arguments(L):
     out = _abi.CalibOut()
     assert L.sq_calib_finish(None, ctypes.byref(budget), ctypes.byref(out), None) == _abi.SQ_ERR_INVALID_ARG
     assert L.sq_calib_free(None) == _abi.SQ_OK
+
+
+def test_prefill_rejects_null_handle_and_negative_sizes(L):
+    P = [None] * 11
+    assert L.sq_prefill(None, *P, 1, 4, None) == _abi.SQ_ERR_INVALID_ARG
+    assert "handle" in L.sq_last_error().decode()
