@@ -9,9 +9,10 @@ columns x20 (synthetic, seeded). One step = one decode step of every
 (request, head) state tile = one launch of the fused kernel.
 
 Prints one JSON line (rank 0). ``value`` is (request*head)-steps/s over all
-ranks with inputs resident in HBM; ``e2e`` is the same through the public
-API with the step's activations copied from pinned host memory and o copied
-back inside the timed region; ``roofline`` compares the kernel's algorithmic
+ranks with inputs resident in HBM; ``e2e`` is the same through the C ABI's
+host-buffer step (sq_decode_step_host): the step's activations are copied
+from pinned host memory inside the call, overlapping the previous step, and
+o is written into pinned host memory, all inside the timed region; ``roofline`` compares the kernel's algorithmic
 state bytes (codes + row scales + pivots, read and written once) per launch
 with the measured HBM copy bandwidth; ``cpu_baseline`` times the CPU oracle
 on a bounded sample of the same workload.
@@ -201,26 +202,22 @@ def run_ours(args, rank, world, local_rank):
     total_ms = max_over_ranks(total_ms)
     kern_ms = statistics.mean(per_ms)
     # ---- end to end through the public API: pinned host activations in, o out
+    # (sq_decode_step_host: the step's inputs are copied from page-locked host
+    # memory inside the call, overlapping the previous step; o is written
+    # into page-locked host memory by the kernel)
     pinned = [[torch.from_numpy(x).pin_memory() for x in xs] for xs in host_inputs]
     o_host = torch.empty((B, c.h_v, c.d), dtype=torch.float32).pin_memory()
-    staging = [torch.empty_like(x) for x in dev_inputs[0]]
     h2d = sum(x.numel() * x.element_size() for x in pinned[0])
     d2h = o_host.numel() * o_host.element_size()
     for i in range(args.warmup):
-        for dst, src in zip(staging, pinned[i % NI]):
-            dst.copy_(src, non_blocking=True)
-        sp.decode_step(pool, *staging, o)
-        o_host.copy_(o, non_blocking=True)
+        sp.decode_step_host(pool, *pinned[i % NI], o_host)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        for dst, src in zip(staging, pinned[i % NI]):
-            dst.copy_(src, non_blocking=True)
-        sp.decode_step(pool, *staging, o)
-        o_host.copy_(o, non_blocking=True)
+        sp.decode_step_host(pool, *pinned[i % NI], o_host)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))

@@ -149,6 +149,30 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
                          const float* beta, const float* g, float* o, const int32_t* slot_ids,
                          int32_t B, void* stream);
 
+/* The same decode step with the activations in HOST memory, for a caller
+ * that keeps them there (the method's paper has no counterpart; this is the
+ * serving loop's host-to-device boundary). q, k, v, beta, g and slot_ids
+ * (or NULL) are host arrays of the shapes of sq_decode_step; o is a host
+ * array [B, h_v, d] written by the step.
+ *   - The inputs are copied on an internal stream into one of two device
+ *     staging sets owned by the handle (allocated at the first call and
+ *     whenever B grows, which synchronizes the device); the copies of a call
+ *     wait only for the step that last used the same set, so they overlap
+ *     the step of the previous call. The step itself runs on `stream` after
+ *     its copies. Page-locked inputs make the copies asynchronous; pageable
+ *     ones are accepted but the copies then block the host.
+ *   - o in mapped page-locked memory (cudaHostAlloc, cudaMallocHost, or
+ *     registered memory on a system with unified addressing) is written by
+ *     the kernel directly over the bus; any other o is staged and copied
+ *     back on `stream`.
+ *   - The host inputs must stay unchanged, and o must not be read, until
+ *     `stream` has passed this call (e.g. cudaStreamSynchronize).
+ * Every step of one handle, device- or host-buffer, must run on one stream
+ * (or streams the caller orders), as for sq_decode_step. */
+sq_status sq_decode_step_host(sq_handle* h, void* pool, const float* q, const float* k, const float* v,
+                              const float* beta, const float* g, float* o, const int32_t* slot_ids, int32_t B,
+                              void* stream);
+
 /* Expand B pool slots to fp32 S [B, h_v, d, d] (device): S_ij = (q r) c_j for
  * quantized rows and h c_j for pivot rows. Skipped (bad) slots give 0. */
 sq_status sq_dequantize_state(sq_handle* h, const void* pool, float* S_out, const int32_t* slot_ids,

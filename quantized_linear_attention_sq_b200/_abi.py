@@ -98,6 +98,7 @@ def lib() -> ctypes.CDLL:
     L.sq_decode_step_noalloc.argtypes = [ctypes.POINTER(StateDesc), ctypes.POINTER(Calib)] + [P] * 8 + [I32, P, P]
     L.sq_decode_step_noalloc.restype = ctypes.c_int
     L.sq_prefill.argtypes = [P] * 12 + [I32, I32, P]
+    L.sq_decode_step_host.argtypes = [P, P, P, P, P, P, P, P, P, I32, P]
     L.sq_calib_begin.argtypes = [ctypes.POINTER(StateDesc), P, ctypes.POINTER(P)]
     L.sq_calib_add_states.argtypes = [P, P, I32, P]
     L.sq_calib_add_tokens.argtypes = [P, P, P, I32, P]
@@ -105,7 +106,7 @@ def lib() -> ctypes.CDLL:
     L.sq_calib_free.argtypes = [P]
     for name in ("sq_state_alloc", "sq_state_free", "sq_quantize_state", "sq_decode_step",
                  "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status",
-                 "sq_prefill", "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
+                 "sq_prefill", "sq_decode_step_host", "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
                  "sq_calib_free"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -144,6 +145,10 @@ def sq_quantize_state(h, pool: int, S: int, slot_ids: int | None, B: int, stream
 
 def sq_decode_step(h, pool, q, k, v, beta, g, o, slot_ids, B, stream) -> None:
     check(lib().sq_decode_step(h, pool, q, k, v, beta, g, o, slot_ids, B, stream))
+
+
+def sq_decode_step_host(h, pool, q, k, v, beta, g, o, slot_ids, B, stream) -> None:
+    check(lib().sq_decode_step_host(h, pool, q, k, v, beta, g, o, slot_ids, B, stream))
 
 
 def sq_prefill(h, pool, S0, q, k, v, beta, g, o, S_out, lengths, slot_ids, B, L, stream) -> None:

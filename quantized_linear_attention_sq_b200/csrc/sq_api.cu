@@ -74,6 +74,18 @@ struct sq_handle {
   uint64_t stage_rec = 0;  // largest record that goes through a stage
   size_t step_smem = 0;
   uint64_t launches = 0;
+  // sq_decode_step_host: two device staging sets used in turn, the internal
+  // stream their host-to-device copies run on, and the events that order
+  // the copies after the step that last read a set.
+  struct HostStage {
+    void* block = nullptr;
+    int32_t cap_B = 0;
+    cudaEvent_t copied = nullptr;  // the set's inputs are on the device
+    cudaEvent_t read = nullptr;    // the step that used the set has run
+  };
+  HostStage host_stage[2];
+  cudaStream_t copy_stream = nullptr;
+  uint64_t host_calls = 0;
 };
 
 namespace {
@@ -243,6 +255,42 @@ sq_status validate_desc(const sq_state_desc* d) {
 
 }  // namespace
 
+namespace {
+
+// Launch the decode step on device pointers (already validated).
+sq_status launch_step(sq_handle* h, void* pool, const float* q, const float* k, const float* v, const float* beta,
+                      const float* g, float* o, const int32_t* slot_ids, int32_t B, void* stream) {
+  sqk::StepArgs a{};
+  a.pool = static_cast<uint8_t*>(pool);
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
+  a.slots = slot_ids;
+  a.B = B; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots; a.gate_kind = h->desc.gate;
+  a.nstage = h->nstage; a.rec_cap = h->rec_cap; a.stage_bytes = h->stage_bytes;
+  a.chunk = kStepChunk;
+  a.slot_bytes = h->slot_bytes;
+  a.t = h->tables;
+  const int n_tiles = B * h->desc.h_v;
+  const int grid = n_tiles < h->step_grid ? n_tiles : h->step_grid;
+  const int nt = threads_of(h->d);
+  cudaStream_t st = as_stream(stream);
+  const bool packed = h->desc.fmt == SQ_FMT_PACKED;
+  if (packed) {
+    if (h->d == 128) sqk::k_decode_step_packed<128><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step_packed<64><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step_packed<32><<<grid, nt, h->step_smem, st>>>(a);
+  } else {
+    if (h->d == 128) sqk::k_decode_step_fp32<128><<<grid, nt, h->step_smem, st>>>(a);
+    else if (h->d == 64) sqk::k_decode_step_fp32<64><<<grid, nt, h->step_smem, st>>>(a);
+    else sqk::k_decode_step_fp32<32><<<grid, nt, h->step_smem, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching the decode step");
+  h->launches++;
+  return SQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* sq_last_error(void) { return g_last_error.c_str(); }
@@ -396,6 +444,12 @@ sq_status sq_state_free(sq_handle* h) {
   g_last_error.clear();
   if (!h) return SQ_OK;
   cudaError_t e = cudaDeviceSynchronize();
+  for (auto& hs : h->host_stage) {
+    if (hs.block) cudaFree(hs.block);
+    if (hs.copied) cudaEventDestroy(hs.copied);
+    if (hs.read) cudaEventDestroy(hs.read);
+  }
+  if (h->copy_stream) cudaStreamDestroy(h->copy_stream);
   cudaError_t e2 = cudaFree(h->dev_block);
   delete h;
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
@@ -464,32 +518,83 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
   if ((reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
     return fail(SQ_ERR_INVALID_ARG, "beta/g not 4-byte aligned");
   if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
-  sqk::StepArgs a{};
-  a.pool = static_cast<uint8_t*>(pool);
-  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
-  a.slots = slot_ids;
-  a.B = B; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots; a.gate_kind = h->desc.gate;
-  a.nstage = h->nstage; a.rec_cap = h->rec_cap; a.stage_bytes = h->stage_bytes;
-  a.chunk = kStepChunk;
-  a.slot_bytes = h->slot_bytes;
-  a.t = h->tables;
-  const int n_tiles = B * h->desc.h_v;
-  const int grid = n_tiles < h->step_grid ? n_tiles : h->step_grid;
-  const int nt = threads_of(h->d);
+  return launch_step(h, pool, q, k, v, beta, g, o, slot_ids, B, stream);
+}
+
+
+sq_status sq_decode_step_host(sq_handle* h, void* pool, const float* q, const float* k, const float* v,
+                              const float* beta, const float* g, float* o, const int32_t* slot_ids, int32_t B,
+                              void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (B == 0) return SQ_OK;
+  if ((int64_t)B * h->desc.h_v > (int64_t)INT32_MAX / 2) return fail(SQ_ERR_INVALID_ARG, "B too large");
+  SQ_CHECK_PTR(pool, "pool");
+  if (!q || !k || !v || !beta || !g || !o) return fail(SQ_ERR_INVALID_ARG, "q, k, v, beta, g and o are required");
+  const size_t d = (size_t)h->d, hv = (size_t)h->desc.h_v, hk = (size_t)h->desc.h_k, nB = (size_t)B;
+  const size_t b_qk = 4 * nB * hk * d, b_v = 4 * nB * hv * d, b_beta = 4 * nB * hv;
+  const size_t b_g = h->desc.gate == SQ_GATE_KEY_CHANNEL ? b_v : b_beta, b_slot = 4 * nB;
   cudaStream_t st = as_stream(stream);
-  const bool packed = h->desc.fmt == SQ_FMT_PACKED;
-  if (packed) {
-    if (h->d == 128) sqk::k_decode_step_packed<128><<<grid, nt, h->step_smem, st>>>(a);
-    else if (h->d == 64) sqk::k_decode_step_packed<64><<<grid, nt, h->step_smem, st>>>(a);
-    else sqk::k_decode_step_packed<32><<<grid, nt, h->step_smem, st>>>(a);
-  } else {
-    if (h->d == 128) sqk::k_decode_step_fp32<128><<<grid, nt, h->step_smem, st>>>(a);
-    else if (h->d == 64) sqk::k_decode_step_fp32<64><<<grid, nt, h->step_smem, st>>>(a);
-    else sqk::k_decode_step_fp32<32><<<grid, nt, h->step_smem, st>>>(a);
+  cudaError_t e;
+  if (!h->copy_stream) {
+    if ((e = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags");
+    for (auto& hs : h->host_stage)
+      if ((e = cudaEventCreateWithFlags(&hs.copied, cudaEventDisableTiming)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&hs.read, cudaEventDisableTiming)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventCreateWithFlags");
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launching the decode step");
-  h->launches++;
+  sq_handle::HostStage& hs = h->host_stage[h->host_calls & 1];
+  // staging layout: q | k | v | o | beta | g | slot ids, 256-byte aligned pieces
+  const size_t o_q = 0, o_k = round_up(b_qk, 256), o_v = o_k + round_up(b_qk, 256);
+  const size_t o_o = o_v + round_up(b_v, 256), o_b = o_o + round_up(b_v, 256);
+  const size_t o_g = o_b + round_up(b_beta, 256), o_s = o_g + round_up(b_g, 256);
+  const size_t total = o_s + round_up(b_slot, 256);
+  if (hs.cap_B < B) {
+    // a larger batch than before: wait for every use of the old set, then replace it
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    if (hs.block) cudaFree(hs.block);
+    hs.block = nullptr;
+    hs.cap_B = 0;
+    if ((e = cudaMalloc(&hs.block, total)) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return fail(SQ_ERR_OOM, "cudaMalloc of %zu bytes of staging failed", total);
+    }
+    hs.cap_B = B;
+  }
+  uint8_t* base = static_cast<uint8_t*>(hs.block);
+  float* dq = reinterpret_cast<float*>(base + o_q);
+  float* dk = reinterpret_cast<float*>(base + o_k);
+  float* dv = reinterpret_cast<float*>(base + o_v);
+  float* dout = reinterpret_cast<float*>(base + o_o);
+  float* dbeta = reinterpret_cast<float*>(base + o_b);
+  float* dg = reinterpret_cast<float*>(base + o_g);
+  int32_t* dslot = slot_ids ? reinterpret_cast<int32_t*>(base + o_s) : nullptr;
+  // the copies of this step wait only for the step that last read this set,
+  // so they overlap the step launched by the previous call
+  cudaStream_t cs = h->copy_stream;
+  if ((e = cudaStreamWaitEvent(cs, hs.read, 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dq, q, b_qk, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dk, k, b_qk, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dv, v, b_v, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dbeta, beta, b_beta, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(dg, g, b_g, cudaMemcpyHostToDevice, cs)) != cudaSuccess ||
+      (slot_ids && (e = cudaMemcpyAsync(dslot, slot_ids, b_slot, cudaMemcpyHostToDevice, cs)) != cudaSuccess) ||
+      (e = cudaEventRecord(hs.copied, cs)) != cudaSuccess || (e = cudaStreamWaitEvent(st, hs.copied, 0)) != cudaSuccess)
+    return cuda_fail(e, "staging the step's inputs");
+  // o: written by the kernel straight into mapped page-locked host memory,
+  // else staged and copied back on the caller's stream
+  void* mapped = nullptr;
+  const bool zero_copy = cudaHostGetDevicePointer(&mapped, o, 0) == cudaSuccess && mapped;
+  if (!zero_copy) (void)cudaGetLastError();
+  float* o_dev = zero_copy ? static_cast<float*>(mapped) : dout;
+  sq_status s = launch_step(h, pool, dq, dk, dv, dbeta, dg, o_dev, dslot, B, stream);
+  if (s != SQ_OK) return s;
+  if ((e = cudaEventRecord(hs.read, st)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if (!zero_copy && (e = cudaMemcpyAsync(o, dout, b_v, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail(e, "copying o to the host");
+  h->host_calls++;
   return SQ_OK;
 }
 

@@ -37,6 +37,20 @@ def _ptr(t: torch.Tensor | None, dtype=None, name="tensor", numel=None) -> int |
     return t.data_ptr()
 
 
+def _host_ptr(t: torch.Tensor | None, dtype, name, numel) -> int | None:
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    return t.data_ptr()
+
+
 class StatePool:
     """A layer's recurrent-state pool handle (calibration tables on device).
 
@@ -109,6 +123,22 @@ class StatePool:
                             _ptr(v, torch.float32, "v", B * hv * d), _ptr(beta, torch.float32, "beta", B * hv),
                             _ptr(g, torch.float32, "g", gn), _ptr(o, torch.float32, "o", B * hv * d),
                             _ptr(slot_ids, torch.int32, "slot_ids", B), B, _stream(stream))
+
+    def decode_step_host(self, pool, q, k, v, beta, g, o, slot_ids=None, stream=None):
+        """The decode step with q, k, v, beta, g, slot_ids and o as CPU tensors
+        (page-locked for overlapped copies; o page-locked is written by the
+        kernel directly). The pool stays on the GPU. Read o after the stream
+        has passed the call."""
+        B = q.shape[0]
+        d, hv, hk = self.d, self.h_v, self.h_k
+        gn = B * hv * (d if self.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1)
+        _abi.sq_decode_step_host(self._h, self._check_pool(pool),
+                                 _host_ptr(q, torch.float32, "q", B * hk * d),
+                                 _host_ptr(k, torch.float32, "k", B * hk * d),
+                                 _host_ptr(v, torch.float32, "v", B * hv * d),
+                                 _host_ptr(beta, torch.float32, "beta", B * hv),
+                                 _host_ptr(g, torch.float32, "g", gn), _host_ptr(o, torch.float32, "o", B * hv * d),
+                                 _host_ptr(slot_ids, torch.int32, "slot_ids", B), B, _stream(stream))
 
     def prefill(self, pool, q, k, v, beta, g, o, S0=None, S_out=None, lengths=None, slot_ids=None, stream=None):
         """Run the prompt (q, k [B, L, h_k, d]; v, o [B, L, h_v, d]; beta [B, L, h_v];

@@ -135,3 +135,9 @@ def test_prefill_rejects_null_handle_and_negative_sizes(L):
     P = [None] * 11
     assert L.sq_prefill(None, *P, 1, 4, None) == _abi.SQ_ERR_INVALID_ARG
     assert "handle" in L.sq_last_error().decode()
+
+
+def test_host_step_rejects_bad_arguments_on_the_host(L):
+    assert L.sq_decode_step_host(None, None, None, None, None, None, None, None, None, 1, None) == \
+        _abi.SQ_ERR_INVALID_ARG
+    assert "handle" in L.sq_last_error().decode()
