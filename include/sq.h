@@ -97,7 +97,7 @@ typedef struct {
   const int8_t* unit_bits;    /* [h_v] or [h_v*d_k]; 2, 4, 6 or 8 */
   const uint8_t* pivot_mask;  /* same shape; nonzero = FP16 pivot unit (overrides unit_bits) */
   const float* col_scale;     /* [h_v*d_v] c_j, finite and > 0 */
-  const float* row_impact;    /* [h_v*d_k] phi_i, finite and > 0 */
+  const float* row_impact;    /* [h_v*d_k] phi_i, finite and > 0; used as the clip ratio min(phi_i, 1) */
 } sq_calib;
 
 typedef struct sq_handle sq_handle;

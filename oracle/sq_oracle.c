@@ -49,7 +49,7 @@
  *      one rounding of the exact gated value plus the rounded update)
  *   5. O_j   = sum_i T'_ij q_i (exact, rounded once); o_j = fp32(c_j O_j)
  *   6. m_i   = max_j |T'_ij| (a NaN makes m_i NaN)
- *   7. s_i   = fp32(fp32(phi_i m_i) / qmax_i); r'_i = fp16 of s_i rounded
+ *   7. s_i   = fp32(fp32(min(phi_i, 1) m_i) / qmax_i); r'_i = fp16 of s_i rounded
  *      toward +inf (saturating at 65504); ir_i = 0 if r'_i == 0 else
  *      fp32(1 / r'_i)
  *   8. q'_ij = min(max(RNE(T'_ij * ir_i), -qmax), qmax), the product taken
@@ -276,8 +276,10 @@ static uint32_t store_T(const sqo_desc *D, int h, uint8_t *rec, const float *T) 
       for (int j = 0; j < d; j++) sqo_put_code(row, b, j, 0);
       continue;
     }
-    /* 8. row scale from magnitude x row impact, rounded up to fp16 */
-    float s = (phi[i] * m) / (float)qm;
+    /* 8. row scale from magnitude x row impact, rounded up to fp16; the
+     * impact factor only ever shrinks the scale (a clip ratio, min(phi, 1)) */
+    float clip = phi[i] < 1.0f ? phi[i] : 1.0f;
+    float s = (clip * m) / (float)qm;
     uint16_t rb;
     if (s > 65504.0f) { rb = 0x7bff; st |= ST_SATURATED; }
     else rb = sqo_f16_ru(s);

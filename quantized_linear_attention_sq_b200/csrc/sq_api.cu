@@ -47,6 +47,14 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 uint64_t round_up(uint64_t x, uint64_t m) { return (x + m - 1) / m * m; }
 
+// The row-impact factor as the kernels use it: a clip ratio min(phi, 1).
+// A factor above 1 would set a row scale beyond what the row's largest
+// entry needs; rounding that entry to a code can then give back a larger
+// value, and since the next step's scale is taken from it, the row grows
+// step after step. Capped at 1, the factor only ever clips rows whose
+// measured impact on the readout is low.
+inline float clip_ratio(float phi) { return phi < 1.0f ? phi : 1.0f; }
+
 // Tiles per scheduling chunk of the packed step: consecutive tiles of one
 // head run back to back on a CTA; the imbalance at the end is at most one
 // chunk per CTA.
@@ -392,7 +400,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
     col[x] = packed ? calib->col_scale[x] : 1.0f;
     volatile float c = col[x];
     icol[x] = 1.0f / c;  // IEEE single-precision division
-    phi[x] = packed ? calib->row_impact[x] : 1.0f;
+    phi[x] = packed ? clip_ratio(calib->row_impact[x]) : 1.0f;
   }
   memcpy(host.data() + o_row_off, h->row_off.data(), 2 * nhd);
   memcpy(host.data() + o_row_code, h->row_code.data(), nhd);
@@ -881,7 +889,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
     col[x] = calib->col_scale[x];
     volatile float c = col[x];
     icol[x] = 1.0f / c;  // IEEE single-precision division
-    phi[x] = calib->row_impact[x];
+    phi[x] = clip_ratio(calib->row_impact[x]);
   }
   cudaStream_t st = as_stream(stream);
   e = cudaMemcpyAsync(nd->scratch, host, total, cudaMemcpyHostToDevice, st);
