@@ -715,16 +715,24 @@ sq_status sq_prefill(sq_handle* h, void* pool, const float* S0, const float* q, 
   a.slot_bytes = h->slot_bytes;
   a.t = h->tables;
   const int n_tiles = B * h->desc.h_v;
-  const int nt = threads_of(h->d);
   const uint32_t rec = a.fmt_fp32 ? 0u : (uint32_t)h->max_rec;
   cudaStream_t st = as_stream(stream);
-  if (h->d == 128)
-    sqk::k_prefill<128><<<n_tiles, nt, sqk::PrefillSmem<128>::bytes(rec), st>>>(a);
-  else if (h->d == 64)
-    sqk::k_prefill<64><<<n_tiles, nt, sqk::PrefillSmem<64>::bytes(rec), st>>>(a);
-  else
-    sqk::k_prefill<32><<<n_tiles, nt, sqk::PrefillSmem<32>::bytes(rec), st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaSuccess;
+  if (h->d == 128) {
+    const size_t smem = sqk::PrefillSmem<128>::bytes(rec);
+    e = cudaFuncSetAttribute(sqk::k_prefill<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) sqk::k_prefill<128><<<n_tiles, 256, smem, st>>>(a);
+  } else if (h->d == 64) {
+    const size_t smem = sqk::PrefillSmem<64>::bytes(rec);
+    e = cudaFuncSetAttribute(sqk::k_prefill<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) sqk::k_prefill<64><<<n_tiles, 128, smem, st>>>(a);
+  } else {
+    const size_t smem = sqk::PrefillSmem<32>::bytes(rec);
+    e = cudaFuncSetAttribute(sqk::k_prefill<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) sqk::k_prefill<32><<<n_tiles, 64, smem, st>>>(a);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "setting the prefill's shared memory");
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching the prefill");
   h->launches++;
   return SQ_OK;
