@@ -70,6 +70,18 @@ def test_serving_config_full_size_sampled_requests():
     assert gap <= 1e-4  # GPU FP32 warm-up vs oracle FP32 warm-up
 
 
+@pytest.mark.parametrize("cid,reqs", [(1, [0, 21, 42, 63]), (2, [0, 50, 101, 127])])
+def test_layer_configs_full_batch_sampled(cid, reqs):
+    """The GDN layer (batch 64) and KDA layer (batch 128) workloads at full
+    batch, one launch per step over all requests; the oracle follows four
+    sampled requests for 64 steps."""
+    w = synth.workload(cid)
+    stats, rollout = gu.run_parity(w, 64, check_requests=reqs, use_gpu_warmup=True)
+    _report(f"layer cid={cid} full batch", stats, rollout)
+    stats.check()
+    assert rollout <= gu.ROLLOUT_TOL
+
+
 @pytest.mark.parametrize("layer", [0, 7])
 def test_long_rollout_config_sampled(layer):
     """One KDA layer of the 8-layer, batch-256 workload at full batch; two
