@@ -20,7 +20,8 @@
 // reproducible: a_i = r_i g_i; T = q a_i; P_j = sum_i T_ij k_i;
 // u_j = beta (v_j - c_j P_j); w_j = u_j / c_j (as u_j * fl(1/c_j));
 // T' = fma(k_i, w_j, T); o_j = c_j sum_i T'_ij q_i; m_i = max_j |T'_ij|;
-// r'_i = fp16 round-up of (phi_i m_i) / qmax; q' = RNE(clamp(T' * fl(1/r'))).
+// r'_i = fp16 round-up of (phi_i m_i) / qmax; q' = RNE(clamp(T' * fl(1/r'))),
+// with phi_i the clip ratio from the tables.
 // Only the two column sums depend on summation order.
 #pragma once
 
@@ -408,23 +409,31 @@ __device__ __forceinline__ void load_row(const uint8_t* row, uint8_t code, int c
   }
 }
 
-// Requantize one row chunk of T' with inverse scale `ir` and write it back.
-// fma(T', ir, 2^23 + 2^(b-1)) rounds the exact product T' * ir to the
-// nearest integer (ties to even) in the window [2^23, 2^24) where floats
-// are integers; outside that window the value lies beyond the clamp bounds
-// whichever way it rounds, so clamping afterwards gives exactly the clamped
-// nearest integer. The result's low b bits are then the stored field.
+// sign(x) min(|x|, lim) for lim >= 0 (one instruction on sm_100).
+__device__ __forceinline__ float clamp_abs(float x, float lim) {
+  float r;
+  asm("min.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(x), "f"(lim));
+  return r;
+}
+
+// Requantize one row chunk of T' with inverse scale `ir` = fl(1 / r') and
+// write it back. The code is the nearest integer (ties to even) to the exact
+// product T' * ir, clamped to [-qmax, qmax]. The clamp is applied to T'
+// first, at lim = qmax r' (exact in fp32): a |T'| above lim gives a product
+// of at least lim * ir = qmax (1 + e), |e| <= 2^-24, whose nearest integer
+// is qmax, and lim itself gives exactly qmax, so clamping T' to lim and
+// rounding equals rounding and clamping the code. fma(T'c, ir, 2^23 +
+// 2^(b-1)) then rounds the exact product to the nearest integer in the
+// window [2^23, 2^24) where floats are integers, and its low b bits are the
+// stored field.
 template <int B>
-__device__ __forceinline__ void store_row_q(uint8_t* row, int cc, float ir, const float2 (&t)[8]) {
-  const float qm = (float)((1 << (B - 1)) - 1);
+__device__ __forceinline__ void store_row_q(uint8_t* row, int cc, float ir, float lim, const float2 (&t)[8]) {
   const float magic = 8388608.0f + (float)(1 << (B - 1));
-  const float lo = magic - qm, hi = magic + qm;
   uint32_t fb[16];
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    float2 n = __ffma2_rn(t[p], f2(ir), f2(magic));
-    n.x = fminf(fmaxf(n.x, lo), hi);
-    n.y = fminf(fmaxf(n.y, lo), hi);
+    const float2 tc = make_float2(clamp_abs(t[p].x, lim), clamp_abs(t[p].y, lim));
+    const float2 n = __ffma2_rn(tc, f2(ir), f2(magic));
     fb[2 * p] = __float_as_uint(n.x);
     fb[2 * p + 1] = __float_as_uint(n.y);
   }
@@ -528,7 +537,7 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
   for (int r = 1; r < G::RPT; ++r) mm = mine == r ? m[r] : mm;
   const int im = mine * G::NG + rg;
   const int cm = KC ? KC : row_code[im];
-  float ir_m = 0.0f;
+  float ir_m = 0.0f, lim_m = 0.0f;
   uint16_t rbits = 0x3C00;  // pivot rows keep fp16 1.0 in their scale slot
   if (cm != ROW_PIVOT) {
     if (mm != mm) {
@@ -546,6 +555,7 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
       }
       const float R = __half2float(rh);
       ir_m = (R == 0.0f) ? 0.0f : __frcp_rn(R);
+      lim_m = __fmul_rn((float)((1 << (cm - 1)) - 1), R);  // qmax r', exact
       rbits = __half_as_ushort(rh);
     }
   }
@@ -555,6 +565,7 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
 #pragma unroll
   for (int r = 0; r < G::RPT; ++r) {
     const float ir = __shfl_sync(0xffffffffu, ir_m, base + r);
+    const float lim = __shfl_sync(0xffffffffu, lim_m, base + r);
     const int i = r * G::NG + rg;
     const int code = KC ? KC : row_code[i];
     uint8_t* row = rec + row_offset<D, KC>(row_off, i);
@@ -564,10 +575,10 @@ __device__ __forceinline__ uint32_t requant_rows(uint8_t* rec, const uint16_t* r
       store_row_zero(row, code, cc);
     } else {
       switch (code) {
-        case 8: store_row_q<8>(row, cc, ir, T[r]); break;
-        case 6: store_row_q<6>(row, cc, ir, T[r]); break;
-        case 4: store_row_q<4>(row, cc, ir, T[r]); break;
-        default: store_row_q<2>(row, cc, ir, T[r]); break;
+        case 8: store_row_q<8>(row, cc, ir, lim, T[r]); break;
+        case 6: store_row_q<6>(row, cc, ir, lim, T[r]); break;
+        case 4: store_row_q<4>(row, cc, ir, lim, T[r]); break;
+        default: store_row_q<2>(row, cc, ir, lim, T[r]); break;
       }
     }
   }
@@ -1167,7 +1178,7 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
     const int sm = (grp * RB + mine) * G::NG + rg;  // slot
     const int im = KC ? sm : row_perm[sm];           // row
     const int cm = KC ? KC : row_code[im];
-    float ir_m = 0.0f;
+    float ir_m = 0.0f, lim_m = 0.0f;
     if (cm != ROW_PIVOT) {
       uint16_t rbits = 0;
       if (mm == mm) {
@@ -1182,6 +1193,7 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
         }
         const float R = __half2float(rh);
         ir_m = (R == 0.0f) ? 0.0f : __frcp_rn(R);
+        lim_m = __fmul_rn(qm, R);  // qmax r', exact
         rbits = __half_as_ushort(rh);
       }
       if (cc < RB) reinterpret_cast<uint16_t*>(rec)[im] = rbits;
@@ -1191,14 +1203,15 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
+        const float lim = __shfl_sync(0xffffffffu, lim_m, base + u);
         const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
         const int code = KC ? KC : row_code[i];
         uint8_t* row = rec + row_offset<D, KC>(row_off, i);
         switch (code) {
-          case 8: store_row_q<8>(row, cc, ir, T[u]); break;
-          case 6: store_row_q<6>(row, cc, ir, T[u]); break;
-          case 4: store_row_q<4>(row, cc, ir, T[u]); break;
-          case 2: store_row_q<2>(row, cc, ir, T[u]); break;
+          case 8: store_row_q<8>(row, cc, ir, lim, T[u]); break;
+          case 6: store_row_q<6>(row, cc, ir, lim, T[u]); break;
+          case 4: store_row_q<4>(row, cc, ir, lim, T[u]); break;
+          case 2: store_row_q<2>(row, cc, ir, lim, T[u]); break;
           default: st |= store_row_pivot<false>(row, cc, T[u]); break;
         }
       }
@@ -1206,6 +1219,7 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
 #pragma unroll
       for (int u = 0; u < RB; ++u) {
         const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
+        const float lim = __shfl_sync(0xffffffffu, lim_m, base + u);
         const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
         const int code = KC ? KC : row_code[i];
         uint8_t* row = rec + row_offset<D, KC>(row_off, i);
@@ -1216,10 +1230,10 @@ __device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* 
           store_row_zero(row, code, cc);
         } else {
           switch (code) {
-            case 8: store_row_q<8>(row, cc, ir, T[u]); break;
-            case 6: store_row_q<6>(row, cc, ir, T[u]); break;
-            case 4: store_row_q<4>(row, cc, ir, T[u]); break;
-            default: store_row_q<2>(row, cc, ir, T[u]); break;
+            case 8: store_row_q<8>(row, cc, ir, lim, T[u]); break;
+            case 6: store_row_q<6>(row, cc, ir, lim, T[u]); break;
+            case 4: store_row_q<4>(row, cc, ir, lim, T[u]); break;
+            default: store_row_q<2>(row, cc, ir, lim, T[u]); break;
           }
         }
       }
