@@ -54,13 +54,14 @@ struct PrefillSmem {
   static size_t bytes(uint32_t rec_cap) { return REGION + (rec_cap + 15) / 16 * 16 + 7 * D; }
 };
 
-// A 16-byte shared-memory load the compiler may not merge with an earlier
-// load of the same address: the token's k is read once for S^T k and once
-// for the update, and keeping the first reads alive in registers next to the
-// whole state column would overflow the register file.
+// A 16-byte shared-memory load that is neither merged with an earlier load
+// of the same address nor moved ahead of the other such loads: the token's
+// k is read once for S^T k and once for the update, and keeping reads alive
+// in registers next to the state would overflow the 128 registers a thread
+// has at two CTAs per SM.
 __device__ __forceinline__ float4 lds128(const float* p) {
   float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.volatile.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(smem_u32(p)));
   return v;
@@ -139,7 +140,7 @@ __device__ __forceinline__ float column_tree(const float2 (&S2)[Geo<D>::RPT][Geo
 // two column sums need one shuffle each and no barrier (one barrier per
 // chunk of TC tokens hands over the next chunk's vectors).
 template <int D>
-__global__ void __launch_bounds__(Geo<D>::NT, D == 128 ? 1 : 2) k_prefill(const PrefillArgs a) {
+__global__ void __launch_bounds__(Geo<D>::NT, 2) k_prefill(const PrefillArgs a) {
   using G = Geo<D>;
   using M = PrefillSmem<D>;
   constexpr int NQ = G::NG / 4;  // float2 pairs per row slot and thread
