@@ -44,7 +44,7 @@ struct PrefillArgs {
 // and the head's row tables behind it.
 template <int D>
 struct PrefillSmem {
-  static constexpr int TC = 8;                   // tokens per staged chunk
+  static constexpr int TC = 16;                  // tokens per staged chunk
   static constexpr int TOK = 4 * D + 8;          // floats per token: k q v g | beta g0 pad
   static constexpr int CHUNK = TC * TOK;         // floats per chunk buffer
   static constexpr size_t S_BYTES = (size_t)D * D * 4;
@@ -116,19 +116,22 @@ __device__ __forceinline__ float column_tree(const float2 (&S2)[Geo<D>::RPT][Geo
                                              int hh) {
   using G = Geo<D>;
   constexpr int PH = G::NG / 4;  // pairs of row groups per half
+  // r outer, pairs inner: consecutive loads feed PH independent chains
+  float2 p[PH];
+#pragma unroll
+  for (int r = 0; r < G::RPT; ++r)
+#pragma unroll
+    for (int x = 0; x < PH; x += 2) {
+      const float4 kv = lds128(vec + r * G::NG + hh * (G::NG / 2) + 2 * x);
+      const float2 k0 = make_float2(kv.x, kv.y), k1 = make_float2(kv.z, kv.w);
+      p[x] = r == 0 ? __fmul2_rn(S2[r][x], k0) : __ffma2_rn(S2[r][x], k0, p[x]);
+      p[x + 1] = r == 0 ? __fmul2_rn(S2[r][x + 1], k1) : __ffma2_rn(S2[r][x + 1], k1, p[x + 1]);
+    }
   float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int x = 0; x < PH; x += 2) {
-    float2 p0, p1;
-#pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      const float4 kv = lds128(vec + r * G::NG + hh * (G::NG / 2) + 2 * x);
-      const float2 k0 = make_float2(kv.x, kv.y), k1 = make_float2(kv.z, kv.w);
-      p0 = r == 0 ? __fmul2_rn(S2[r][x], k0) : __ffma2_rn(S2[r][x], k0, p0);
-      p1 = r == 0 ? __fmul2_rn(S2[r][x + 1], k1) : __ffma2_rn(S2[r][x + 1], k1, p1);
-    }
-    a01 = __fadd2_rn(a01, p0);
-    a23 = __fadd2_rn(a23, p1);
+    a01 = __fadd2_rn(a01, p[x]);
+    a23 = __fadd2_rn(a23, p[x + 1]);
   }
   const float t = __fadd_rn(__fadd_rn(a01.x, a01.y), __fadd_rn(a23.x, a23.y));
   return __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, 1));  // t0 + t1 on both threads (addition commutes)
