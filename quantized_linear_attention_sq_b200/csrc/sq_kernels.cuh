@@ -1,8 +1,8 @@
 // sq_kernels.cuh -- sm_100a kernels of the quantized-state decode step.
 //
 // One CTA owns one (request, value head) state tile at a time. CTAs are
-// persistent: each walks a contiguous run of tiles, and its records (plus
-// the tile's small vectors and the head's calibration rows) arrive in shared
+// persistent and take tiles in turn (the packed step claims them from a work
+// counter); the records (plus the tile's small vectors and head tables) arrive in shared
 // memory through 1-D TMA bulk copies (cp.async.bulk, no multicast) completed
 // on an mbarrier, NSTAGE tiles ahead of the one being computed. The updated
 // record is written back in place from shared memory with a bulk store. The
