@@ -367,12 +367,14 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     # each of the --steps steps is a bounded sample of the workload; the whole
-    # run is sized to about a minute of CPU time
-    cb = cpu_baseline(args, target_s=60.0, steps=max(1, args.steps))
+    # run is sized to 4 x --cpu-seconds of CPU time (a minute by default)
+    cb = cpu_baseline(args, target_s=4.0 * args.cpu_seconds, steps=max(1, args.steps))
     from quantized_linear_attention_sq_b200 import synth
     w = synth.workload(CONFIG_ID, seed=args.seed)
+    full_step_ms = 1e3 * w.cfg.batch * w.cfg.h_v / cb["value"]  # one whole-batch step at the sample's rate
     out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_step_ms,
+           "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
            "config": workload_config(w), "cpu_baseline": cb,
            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
