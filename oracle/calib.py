@@ -108,8 +108,8 @@ def col_scales(m2: np.ndarray, phi: np.ndarray, n_states: int) -> np.ndarray:
     c = 1."""
     m2 = np.asarray(m2, dtype=np.float64)
     w = np.asarray(phi, dtype=np.float64) ** 2
-    h_v, d, _ = m2.shape
-    out = np.ones((h_v, d), dtype=np.float64)
+    h_v, _, n_cols = m2.shape
+    out = np.ones((h_v, n_cols), dtype=np.float64)
     for h in range(h_v):
         num = (w[h][:, None] * m2[h]).sum(axis=0)
         rho = np.sqrt(num / (n_states * w[h].sum()))
