@@ -99,6 +99,15 @@ sq_status sq_calib_add_tokens(sq_calib_trace* t, const float* q, const float* g,
 sq_status sq_calib_finish(sq_calib_trace* t, const sq_calib_budget* budget, const sq_calib_out* out,
                           void* stream);
 
+/* The width allocation alone, on the host (no device work): the widths and
+ * FP16 pivots sq_calib_finish chooses for N units with mean squares
+ * sigma2[N] and lifetime weights weight[N] (host arrays, finite and >= 0)
+ * under `budget` (rules in the header comment above). For callers that
+ * compute the unit statistics themselves. unit_bits and pivot_mask are host
+ * arrays of N entries. */
+sq_status sq_calib_allocate(const double* sigma2, const double* weight, int64_t n, const sq_calib_budget* budget,
+                            int8_t* unit_bits, uint8_t* pivot_mask);
+
 /* Release the trace (synchronizes the device first). NULL is a no-op. */
 sq_status sq_calib_free(sq_calib_trace* t);
 

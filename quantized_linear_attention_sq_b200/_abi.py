@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
     L.sq_decode_step_noalloc.restype = ctypes.c_int
     L.sq_prefill.argtypes = [P] * 12 + [I32, I32, P]
     L.sq_decode_step_host.argtypes = [P, P, P, P, P, P, P, P, P, I32, P]
+    L.sq_calib_allocate.argtypes = [P, P, ctypes.c_int64, ctypes.POINTER(CalibBudget), P, P]
     L.sq_calib_begin.argtypes = [ctypes.POINTER(StateDesc), P, ctypes.POINTER(P)]
     L.sq_calib_add_states.argtypes = [P, P, I32, P]
     L.sq_calib_add_tokens.argtypes = [P, P, P, I32, P]
@@ -106,7 +107,7 @@ def lib() -> ctypes.CDLL:
     L.sq_calib_free.argtypes = [P]
     for name in ("sq_state_alloc", "sq_state_free", "sq_quantize_state", "sq_decode_step",
                  "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status",
-                 "sq_prefill", "sq_decode_step_host", "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
+                 "sq_prefill", "sq_decode_step_host", "sq_calib_allocate", "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
                  "sq_calib_free"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -212,3 +213,20 @@ def sq_calib_finish(t, budget: CalibBudget, out: CalibOut, stream: int) -> None:
 
 def sq_calib_free(t) -> None:
     check(lib().sq_calib_free(t))
+
+
+def sq_calib_allocate(sigma2, weight, widths, nominal_bits, pivot_frac):
+    """Host-only width allocation (numpy arrays in, (unit_bits int8, pivot uint8) out)."""
+    import numpy as np
+    s2 = np.ascontiguousarray(sigma2, dtype=np.float64)
+    w = np.ascontiguousarray(weight, dtype=np.float64)
+    n = s2.shape[0]
+    bits = np.zeros(n, np.int8)
+    piv = np.zeros(n, np.uint8)
+    mask = 0
+    for b in widths:
+        mask |= 1 << int(b)
+    check(lib().sq_calib_allocate(s2.ctypes.data, w.ctypes.data, n,
+                                  ctypes.byref(CalibBudget(mask, int(nominal_bits), float(pivot_frac))),
+                                  bits.ctypes.data, piv.ctypes.data))
+    return bits, piv

@@ -269,9 +269,43 @@ void allocate(const std::vector<double>& s2, const std::vector<double>& w, const
   }
 }
 
+// The allowed widths of a budget, ascending, after checking the budget.
+sq_status check_budget(const sq_calib_budget* budget, std::vector<int>& widths) {
+  widths.clear();
+  for (int b = 0; b < 31; ++b) {
+    if (!(budget->widths_mask >> b & 1)) continue;
+    if (b != 2 && b != 4 && b != 6 && b != 8) return fail(SQ_ERR_INVALID_ARG, "width %d not in {2,4,6,8}", b);
+    widths.push_back(b);
+  }
+  if (widths.empty()) return fail(SQ_ERR_INVALID_ARG, "widths_mask allows no width");
+  if (budget->nominal_bits < widths.front() || budget->nominal_bits > widths.back())
+    return fail(SQ_ERR_INVALID_ARG, "nominal_bits %d outside [%d, %d]", budget->nominal_bits, widths.front(),
+                widths.back());
+  if (!(budget->pivot_frac >= 0.0 && budget->pivot_frac <= 1.0))
+    return fail(SQ_ERR_INVALID_ARG, "pivot_frac must be in [0, 1]");
+  return SQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+sq_status sq_calib_allocate(const double* sigma2, const double* weight, int64_t n, const sq_calib_budget* budget,
+                            int8_t* unit_bits, uint8_t* pivot_mask) {
+  sqi::g_last_error.clear();
+  if (!budget || n < 0) return fail(SQ_ERR_INVALID_ARG, "budget must not be NULL and n must be >= 0");
+  if (n > 0 && (!sigma2 || !weight || !unit_bits || !pivot_mask))
+    return fail(SQ_ERR_INVALID_ARG, "sigma2, weight, unit_bits and pivot_mask are required");
+  std::vector<int> widths;
+  const sq_status bs = check_budget(budget, widths);
+  if (bs != SQ_OK) return bs;
+  std::vector<double> s2(sigma2, sigma2 + n), w(weight, weight + n);
+  for (int64_t u = 0; u < n; ++u)
+    if (!(std::isfinite(s2[u]) && s2[u] >= 0.0 && std::isfinite(w[u]) && w[u] >= 0.0))
+      return fail(SQ_ERR_INVALID_ARG, "unit %lld: sigma2 and weight must be finite and >= 0", (long long)u);
+  allocate(s2, w, widths, budget->nominal_bits, budget->pivot_frac, unit_bits, pivot_mask);
+  return SQ_OK;
+}
 
 sq_status sq_calib_begin(const sq_state_desc* desc, void* stream, sq_calib_trace** out) {
   sqi::g_last_error.clear();
@@ -369,17 +403,8 @@ sq_status sq_calib_finish(sq_calib_trace* t, const sq_calib_budget* budget, cons
   if (t->n_states == 0 || t->n_q == 0 || t->n_g == 0)
     return fail(SQ_ERR_INVALID_ARG, "finish needs at least one state, one query and one gate sample");
   std::vector<int> widths;
-  for (int b = 0; b < 31; ++b) {
-    if (!(budget->widths_mask >> b & 1)) continue;
-    if (b != 2 && b != 4 && b != 6 && b != 8) return fail(SQ_ERR_INVALID_ARG, "width %d not in {2,4,6,8}", b);
-    widths.push_back(b);
-  }
-  if (widths.empty()) return fail(SQ_ERR_INVALID_ARG, "widths_mask allows no width");
-  if (budget->nominal_bits < widths.front() || budget->nominal_bits > widths.back())
-    return fail(SQ_ERR_INVALID_ARG, "nominal_bits %d outside [%d, %d]", budget->nominal_bits, widths.front(),
-                widths.back());
-  if (!(budget->pivot_frac >= 0.0 && budget->pivot_frac <= 1.0))
-    return fail(SQ_ERR_INVALID_ARG, "pivot_frac must be in [0, 1]");
+  const sq_status bs = check_budget(budget, widths);
+  if (bs != SQ_OK) return bs;
 
   cudaStream_t st = as_stream(stream);
   const int per_row = t->gate == SQ_GATE_KEY_CHANNEL;

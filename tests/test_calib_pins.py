@@ -187,3 +187,52 @@ def test_calibrate_from_trace_constant_tokens_matches_direct():
     b = oc.calibrate(states, qrow.astype(np.float64) ** 2, grow, False, (4, 6, 8), 6, 0.0)
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
+
+
+# ---------------------------------------------------------------------------
+# The library's width allocation (sq_calib_allocate, host code in the CUDA
+# library) against the oracle's, exactly: the same widths and pivots.
+
+def _lib_alloc(sigma2, w, widths, nominal, pf):
+    from quantized_linear_attention_sq_b200 import _abi, build
+    build.build()
+    return _abi.sq_calib_allocate(sigma2, w, widths, nominal, pf)
+
+
+@pytest.mark.parametrize("seed,n,widths,nominal,pf", [
+    (0, 32, (4, 6, 8), 6, 0.05),        # GDN layer: units are heads
+    (1, 512, (2, 4, 6), 4, 0.03),       # KDA: units are key rows
+    (2, 513, (2, 4, 6, 8), 5, 0.0),     # odd count, all four widths
+    (3, 300, (4, 8), 6, 0.1),           # unequal raise sizes (4 -> 8)
+    (4, 64, (2, 8), 2, 1.0),            # every unit a pivot
+])
+def test_library_allocation_equals_oracle(seed, n, widths, nominal, pf):
+    rng = np.random.default_rng(seed)
+    sigma2 = rng.lognormal(0.0, 1.5, size=n)
+    w = 1.0 / (1.0 - rng.uniform(0.0, 0.999, size=n))
+    want_bits, want_piv = oc.allocate(sigma2, w, widths, nominal, pf)
+    got_bits, got_piv = _lib_alloc(sigma2, w, widths, nominal, pf)
+    np.testing.assert_array_equal(got_piv, want_piv)
+    np.testing.assert_array_equal(got_bits, want_bits)
+
+
+def test_library_allocation_ties_go_to_the_lower_index():
+    # identical units, zero-variance units and repeated distortions: every
+    # tie is decided by the unit index on both sides
+    sigma2 = np.array([1.0, 1.0, 0.0, 2.0, 2.0, 0.0, 1.0, 2.0] * 8)
+    w = np.array([1.0, 1.0, 3.0, 0.5, 0.5, 1.0, 1.0, 0.5] * 8)
+    for widths, nominal, pf in (((2, 4, 6, 8), 5, 0.1), ((4, 6, 8), 6, 0.0), ((2, 4), 3, 0.25)):
+        want = oc.allocate(sigma2, w, widths, nominal, pf)
+        got = _lib_alloc(sigma2, w, widths, nominal, pf)
+        np.testing.assert_array_equal(got[1], want[1])
+        np.testing.assert_array_equal(got[0], want[0])
+
+
+def test_library_allocation_rejects_bad_budgets_and_values():
+    from quantized_linear_attention_sq_b200 import _abi
+    s = np.ones(4)
+    for widths, nominal, pf in (((3, 4), 4, 0.0), ((4, 6), 8, 0.0), ((4, 6), 5, 1.5), ((), 4, 0.0)):
+        with pytest.raises(_abi.SQError):
+            _lib_alloc(s, s, widths, nominal, pf)
+    with pytest.raises(_abi.SQError, match="finite"):
+        _lib_alloc(np.array([1.0, np.nan, 1.0, 1.0]), s, (4, 6), 5, 0.0)
