@@ -6,14 +6,17 @@ its binding in ``quantized_linear_attention_sq_b200``) never does: it shares
 no code with the oracle and fails loudly when its own extension is missing.
 
 The arithmetic lives in ``sq_oracle.c`` (plain C, fp32 elementwise steps in
-the order the method states them, fp64-accumulated dot products). This
+the order the method states them; every column dot product is summed exactly
+in a fixed-point accumulator and rounded once to fp32). This
 module only marshals numpy arrays into it. See the header of ``sq_oracle.c``
 for the definition of every step and of the storage format.
 
 Parity pins (tests/test_oracle_pins.py) tie it to the textbook gated delta
 rule, the delta-rule invariant, closed forms, Proposition 1 of the method,
 the quantizer error bound, brute force over all codes and all fp16 values,
-and the bit accounting printed for Table D3 of the method's paper.
+and the bit accounting printed for Table D3 of the method's paper;
+tests/test_exact_sum_pins.py ties the exact column sums to a second exact
+computation on columns built to sit next to fp32 rounding boundaries.
 """
 from __future__ import annotations
 

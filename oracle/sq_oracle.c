@@ -31,10 +31,15 @@
  * The pages fix the method but not its arithmetic; the canonical
  * elementwise arithmetic below is this project's reading, chosen so that
  * two implementations agree bit for bit on the integer codes. The only sums
- * are the two column dot products; each is taken from exact products and
- * rounded once to fp32 (here: exact products and an extended-precision
- * accumulator). S^T k is the one sum that feeds back into the state, so it
- * is the one whose rounding decides reproducibility over a long rollout.
+ * are the column dot products (S^T k and S^T q); each is the exact value of
+ * the sum of exact products, rounded once to fp32 (round to nearest, ties to
+ * even; an exact zero gives +0). Here that is computed literally: every
+ * product is an integer times a power of two, and the products are added
+ * without rounding in a wide fixed-point accumulator (xacc below) that is
+ * rounded once at the end. S^T k is the one sum that feeds back into the
+ * state, so it is the one whose rounding decides reproducibility over a
+ * long rollout; because it is exact, the result does not depend on any
+ * summation order.
  *
  * Column-normalised form. With S = T diag(c), the whole step is carried out
  * on T (the row-scale x code part), and c enters only where S^T k and S^T q
@@ -153,6 +158,113 @@ uint16_t sqo_f16_ru(float x) {
   double t = ldexp(a, -qe);
   double n = sign ? floor(t) : ceil(t); /* toward +inf: down in magnitude for negatives */
   return f16_encode(sign, n, qe);
+}
+
+/* --------------------------------------------------------- exact sums */
+/* A sum of products of floats, held exactly. Every finite float is an
+ * integer significand times a power of two (frexp gives x = f 2^e with
+ * f in [0.5, 1); f 2^24 is an integer for any float, subnormals included),
+ * so a product of up to three floats is an integer below 2^72 times a power
+ * of two. The accumulator is a two's complement fixed-point number of
+ * XA_LIMBS 32-bit limbs whose bit 0 has weight 2^XA_LSB; that covers every
+ * product of three finite floats (smallest weight 2^(3 (-149 - 23)) =
+ * 2^-516, largest below 2^(3 128)) with room for the carries of any
+ * number of terms this file adds. Each limb is kept in an int64 and
+ * normalised only at the end, so adding a term never loses a bit.
+ * A term that is not finite (inf or NaN operand) switches the sum to the
+ * IEEE result, which for such terms does not depend on the order. */
+#define XA_LIMBS 32
+#define XA_LSB (-544)
+
+typedef struct {
+  int64_t limb[XA_LIMBS];
+  int nonfinite;
+  long double ieee; /* IEEE sum, used only when a term is not finite */
+} xacc;
+
+static void xacc_init(xacc *a) { memset(a, 0, sizeof *a); }
+
+/* significand and exponent of a finite float: x = m 2^e exactly, m >= 0 */
+static void split_f32(float x, uint64_t *m, int *e) {
+  int ex;
+  double f = frexp(fabs((double)x), &ex);
+  *m = (uint64_t)ldexp(f, 24);
+  *e = ex - 24;
+}
+
+/* a += x * y * z (pass z = 1 for a product of two) */
+static void xacc_add3(xacc *a, float x, float y, float z) {
+  if (!isfinite(x) || !isfinite(y) || !isfinite(z)) {
+    a->nonfinite = 1;
+    a->ieee += (long double)x * (long double)y * (long double)z;
+    return;
+  }
+  a->ieee += (long double)x * (long double)y * (long double)z;
+  if (x == 0.0f || y == 0.0f || z == 0.0f) return;
+  uint64_t mx, my, mz;
+  int ex, ey, ez;
+  split_f32(x, &mx, &ex);
+  split_f32(y, &my, &ey);
+  split_f32(z, &mz, &ez);
+  unsigned __int128 v = (unsigned __int128)mx * my * mz; /* < 2^72 */
+  int pos = ex + ey + ez - XA_LSB;                       /* bit index of v's bit 0 */
+  int neg = signbit(x) ^ signbit(y) ^ signbit(z);
+  int li = pos / 32, sh = pos % 32;
+  v <<= sh; /* < 2^103 */
+  for (int t = 0; t < 4 && li + t < XA_LIMBS; t++) {
+    int64_t piece = (int64_t)(uint32_t)(v >> (32 * t));
+    a->limb[li + t] += neg ? -piece : piece;
+  }
+}
+
+/* carries into limbs 0 .. XA_LIMBS-2 in [0, 2^32); the top limb keeps the sign */
+static void xacc_normalise(int64_t *l) {
+  for (int i = 0; i + 1 < XA_LIMBS; i++) {
+    int64_t c = l[i] >> 32; /* floor division by 2^32 (arithmetic shift) */
+    l[i] -= c * ((int64_t)1 << 32);
+    l[i + 1] += c;
+  }
+}
+
+static int limb_bit(const int64_t *l, int n) { return (int)((l[n / 32] >> (n % 32)) & 1); }
+
+/* The exact sum rounded once to fp32: to nearest, ties to even, with the
+ * subnormal quantum 2^-149 at the bottom and inf above the largest float;
+ * an exact zero gives +0. */
+static float xacc_round_f32(const xacc *a) {
+  if (a->nonfinite) return (float)a->ieee;
+  int64_t l[XA_LIMBS];
+  memcpy(l, a->limb, sizeof l);
+  xacc_normalise(l);
+  int neg = l[XA_LIMBS - 1] < 0;
+  if (neg) {
+    for (int i = 0; i < XA_LIMBS; i++) l[i] = -l[i];
+    xacc_normalise(l);
+  }
+  int top = -1; /* index of the most significant set bit */
+  for (int n = 32 * XA_LIMBS - 1; n >= 0; n--)
+    if (limb_bit(l, n)) { top = n; break; }
+  if (top < 0) return 0.0f;
+  int qexp = top + XA_LSB - 23; /* exponent of the unit in the last place */
+  if (qexp < -149) qexp = -149;
+  int q0 = qexp - XA_LSB; /* bit index of that unit */
+  uint64_t n = 0;
+  for (int b = top; b >= q0 && b >= 0; b--) n = (n << 1) | (uint64_t)limb_bit(l, b);
+  int half = q0 - 1 >= 0 ? limb_bit(l, q0 - 1) : 0;
+  int sticky = 0;
+  for (int b = q0 - 2; b >= 0 && !sticky; b--) sticky = limb_bit(l, b);
+  if (half && (sticky || (n & 1))) n++;
+  float r = (float)ldexp((double)n, qexp); /* exact, or inf beyond the largest float */
+  return neg ? -r : r;
+}
+
+/* sum_i x[i] y[i] z[i] exactly (z may be NULL: all ones), rounded once; an
+ * entry point of its own so that the pins can check the exact sum directly */
+float sqo_exact_dot3(const float *x, const float *y, const float *z, int n) {
+  xacc a;
+  xacc_init(&a);
+  for (int i = 0; i < n; i++) xacc_add3(&a, x[i], y[i], z ? z[i] : 1.0f);
+  return xacc_round_f32(&a);
 }
 
 /* -------------------------------------------------------------- layout */
@@ -332,10 +444,10 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
 
   load_VM(D, h, rec, gate, T, M);                      /* step 1 */
   for (int j = 0; j < d; j++) {                        /* steps 2-3 */
-    /* each product V * M * k is exact in long double (at most 59 bits) */
-    long double acc = 0.0L;
-    for (int i = 0; i < d; i++) acc += (long double)T[i * d + j] * (long double)M[i] * (long double)k[i];
-    float P = (float)acc;
+    xacc acc;
+    xacc_init(&acc);
+    for (int i = 0; i < d; i++) xacc_add3(&acc, T[i * d + j], M[i], k[i]);
+    float P = xacc_round_f32(&acc);
     float p = c[j] * P;
     float u = beta * (v[j] - p);
     float ic = 1.0f / c[j];
@@ -347,9 +459,10 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
       T[i * d + j] = fmaf(T[i * d + j], M[i], kw);
     }
   for (int j = 0; j < d; j++) {                        /* step 5 */
-    long double acc = 0.0L;
-    for (int i = 0; i < d; i++) acc += (long double)T[i * d + j] * (long double)q[i];
-    float O = (float)acc;
+    xacc acc;
+    xacc_init(&acc);
+    for (int i = 0; i < d; i++) xacc_add3(&acc, T[i * d + j], q[i], 1.0f);
+    float O = xacc_round_f32(&acc);
     o[j] = c[j] * O;
     if (isnan(o[j])) st |= ST_NAN;
   }
@@ -448,7 +561,8 @@ uint32_t sqo_dequantize(const sqo_desc *D, const uint8_t *pool, float *S, const 
 /* Unquantized FP32 state step (S-space) for tiles [t0, t1), S pool
  * [n_slots, h_v, d, d]:
  *   G = g_i S_ij ; P_j = sum_i G_ij k_i ; u_j = beta (v_j - P_j) ;
- *   S'_ij = fmaf(k_i, u_j, G_ij) ; o_j = sum_i S'_ij q_i. */
+ *   S'_ij = fmaf(k_i, u_j, G_ij) ; o_j = sum_i S'_ij q_i,
+ * both sums exact and rounded once, as in the quantized step. */
 uint32_t sqo_step_fp32_tiles(const sqo_desc *D, float *Spool, const float *q_all, const float *k_all,
                              const float *v_all, const float *beta_all, const float *g_all, float *o_all,
                              const int32_t *slots, int t0, int t1) {
@@ -471,17 +585,19 @@ uint32_t sqo_step_fp32_tiles(const sqo_desc *D, float *Spool, const float *q_all
     for (int i = 0; i < d; i++)
       for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
     for (int j = 0; j < d; j++) {
-      long double acc = 0.0L;
-      for (int i = 0; i < d; i++) acc += (long double)S[i * d + j] * (long double)k[i];
-      float P = (float)acc;
+      xacc acc;
+      xacc_init(&acc);
+      for (int i = 0; i < d; i++) xacc_add3(&acc, S[i * d + j], k[i], 1.0f);
+      float P = xacc_round_f32(&acc);
       u[j] = beta * (v[j] - P);
     }
     for (int i = 0; i < d; i++)
       for (int j = 0; j < d; j++) S[i * d + j] = fmaf(k[i], u[j], S[i * d + j]);
     for (int j = 0; j < d; j++) {
-      double acc = 0.0;
-      for (int i = 0; i < d; i++) acc += (double)S[i * d + j] * (double)q[i];
-      o[j] = (float)acc;
+      xacc acc;
+      xacc_init(&acc);
+      for (int i = 0; i < d; i++) xacc_add3(&acc, S[i * d + j], q[i], 1.0f);
+      o[j] = xacc_round_f32(&acc);
       if (isnan(o[j])) st |= ST_NAN;
     }
   }
