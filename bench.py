@@ -148,6 +148,7 @@ def run_ours(args, rank, world, local_rank):
     sp.quantize_state(pool, S)
     torch.cuda.synchronize()
     setup_status = sp.get_status()
+    sp.exact_count(clear=True)
     NI = 8
     host_inputs = [w.step_inputs(t) for t in range(NI)]
     dev_inputs = [[torch.from_numpy(x).to(dev) for x in xs] for xs in host_inputs]
@@ -158,7 +159,8 @@ def run_ours(args, rank, world, local_rank):
             sp.decode_step(pool, *dev_inputs[i % NI], o)
         torch.cuda.synchronize()
         print(json.dumps({"profile_steps": args.profile, "status_after_setup": setup_status,
-                          "status_bits": sp.get_status()}), flush=True)
+                          "status_bits": sp.get_status(), "launch": sp.launch_plan(),
+                          "exact_sum_columns": sp.exact_count()}), flush=True)
         sp.close()
         fp.close()
         return
@@ -222,6 +224,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     st_bits = sp.get_status()
+    exact_cols = sp.exact_count() / (2 * (args.steps + args.warmup))
     # ---- FP32-state step on the same workload (unquantized comparison)
     fp_pool = S  # warmed-up fp32 state, same requests
     fp_total, fp_per, _ = timed_device(fp, fp_pool, max(4, args.steps // 4), args.warmup)
@@ -250,7 +253,8 @@ def run_ours(args, rank, world, local_rank):
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
                   "clip_fraction": clip,
                   "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
-                  "status_bits": st_bits},
+                  "status_bits": st_bits, "exact_sum_columns_per_step": exact_cols},
+        "launch": sp.launch_plan(),
         "fp32_state": {"value": shards.job_rate(units, max(4, args.steps // 4), fp_total, world),
                        "kernel_ms": fp_kern, "achieved_gbs": fp_bytes / (fp_kern / 1e3) / 1e9,
                        "frac": fp_bytes / (fp_kern / 1e3) / 1e9 / peak,

@@ -111,7 +111,9 @@ typedef struct {
   uint64_t max_record_bytes;       /* largest head record */
 } sq_bytes_report;
 
-/* Create a handle: validate the description and calibration, build the
+/* Plumbing (no passage of the method's pages: handle, layout and error
+ * reporting around the steps). Create a handle: validate the description
+ * and calibration, build the
  * record layout and upload the per-head tables (ic_j = 1/c_j included) to
  * the current device with cudaMalloc + cudaMemcpyAsync on `stream`. The
  * state pool itself is NOT allocated: the caller allocates pool_bytes
@@ -121,7 +123,8 @@ typedef struct {
 sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void* stream,
                          sq_handle** out, size_t* pool_bytes);
 
-/* Release the handle's device tables (synchronizes the device first). NULL is a no-op. */
+/* Plumbing (no passage). Release the handle's device tables (synchronizes
+ * the device first). NULL is a no-op. */
 sq_status sq_state_free(sq_handle* h);
 
 /* Quantize B fp32 states into pool slots ("STEPQuant review (e-cogni)",
@@ -206,17 +209,56 @@ sq_status sq_prefill(sq_handle* h, void* pool, const float* S0, const float* q, 
                      const float* beta, const float* g, float* o, float* S_out, const int32_t* lengths,
                      const int32_t* slot_ids, int32_t B, int32_t L, void* stream);
 
-/* Byte accounting of the layout (host only, no device work). */
+/* Byte accounting of the layout (host only, no device work); the per-step
+ * figures are the algorithmic bytes of Table D3's accounting applied to
+ * this layout ("STEPQuant: estados recurrentes a 6 bit" (gpt-diffusion),
+ * section on what the "6-bit" and the "68,7%" mean). */
 sq_status sq_state_bytes(const sq_handle* h, sq_bytes_report* out);
 
-/* Offset within a slot and size of value head `head`'s record (host only). */
+/* Plumbing (no passage). Offset within a slot and size of value head
+ * `head`'s record (host only). */
 sq_status sq_head_layout(const sq_handle* h, int32_t head, uint64_t* offset, uint64_t* record_bytes);
 
-/* Synchronize `stream`, return the device status bits accumulated since the
- * last clear, and clear them if `clear` is nonzero. */
+/* Plumbing (no passage). Synchronize `stream`, return the device status
+ * bits accumulated since the last clear, and clear them if `clear` is
+ * nonzero. */
 sq_status sq_get_status(sq_handle* h, void* stream, uint32_t* bits, int32_t clear);
 
-/* Number of kernel launches this handle has issued (host-side counter). */
+/* Number of columns whose S^T k the packed decode steps of this handle have
+ * summed with the exact fixed-point accumulator since the last clear. The
+ * step defines S^T k as the exact value of the sum rounded once to fp32
+ * (the reading of the quantize-after-every-update loop in "STEPQuant review
+ * (e-cogni)", section "Contexto": the state feeds its own rounding back
+ * every step, so the rounding must not depend on summation order); the
+ * kernel sums in fp64, rounds when a rigorous error bound shows the fp64
+ * total rounds like the exact value, and sums the column exactly otherwise.
+ * This counts the latter (a diagnostic; rare on real data). Synchronizes
+ * `stream`; clears the count if `clear` is nonzero. */
+sq_status sq_get_exact_count(sq_handle* h, void* stream, uint32_t* count, int32_t clear);
+
+/* Plumbing (no passage). Limit, in nanoseconds, of every bounded wait inside
+ * this handle's step kernels (default 2 s; at least 1000). A wait that runs
+ * out abandons its tile before anything of it is written and sets
+ * SQ_STATUS_TIMEOUT. */
+sq_status sq_set_wait_limit(sq_handle* h, uint64_t ns);
+
+/* Testing only (no passage). From the next packed decode step on, CTA 0 of
+ * each launch makes every stage it fills expect `extra_bytes` (at most
+ * 65536) more bytes than it loads, so its first wait runs out after the wait
+ * limit: the step sets SQ_STATUS_TIMEOUT, writes no part of the tiles CTA 0
+ * had taken, and the other CTAs finish the rest. 0 restores normal
+ * operation. Every copy CTA 0 issues still lands; nothing is left in flight. */
+sq_status sq_test_stall_stages(sq_handle* h, uint32_t extra_bytes);
+
+/* Plumbing (no passage). Launch configuration of this handle's decode step
+ * kernel (host only): grid size (persistent CTAs), threads per CTA, CTAs
+ * resident per SM, shared-memory stages per CTA and dynamic shared-memory
+ * bytes per CTA. Any pointer may be NULL. */
+sq_status sq_launch_plan(const sq_handle* h, int32_t* grid, int32_t* threads, int32_t* ctas_per_sm,
+                         int32_t* stages, int32_t* smem_bytes);
+
+/* Plumbing (no passage). Number of kernel launches this handle has issued
+ * (host-side counter). */
 uint64_t sq_launch_count(const sq_handle* h);
 
 /* Decode step that allocates nothing. The method's paper has no
@@ -250,10 +292,11 @@ sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_calib* cali
                                  const float* k, const float* v, const float* beta, const float* g, float* o,
                                  const int32_t* slot_ids, int32_t B, uint32_t* status, void* stream);
 
-/* Message for the last non-OK return on this host thread ("" if none). */
+/* Plumbing (no passage). Message for the last non-OK return on this host
+ * thread ("" if none). */
 const char* sq_last_error(void);
 
-/* Library version string. */
+/* Plumbing (no passage). Library version string. */
 const char* sq_version(void);
 
 #ifdef __cplusplus

@@ -90,6 +90,10 @@ def lib() -> ctypes.CDLL:
     L.sq_head_layout.argtypes = [P, I32, ctypes.POINTER(U64), ctypes.POINTER(U64)]
     L.sq_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32), I32]
     L.sq_launch_count.argtypes = [P]
+    L.sq_get_exact_count.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32), I32]
+    L.sq_set_wait_limit.argtypes = [P, U64]
+    L.sq_launch_plan.argtypes = [P] + [ctypes.POINTER(I32)] * 5
+    L.sq_test_stall_stages.argtypes = [P, ctypes.c_uint32]
     L.sq_launch_count.restype = U64
     L.sq_last_error.argtypes = []
     L.sq_last_error.restype = ctypes.c_char_p
@@ -180,6 +184,26 @@ def sq_get_status(h, stream: int, clear: bool = True) -> int:
 
 def sq_launch_count(h) -> int:
     return int(lib().sq_launch_count(h))
+
+
+def sq_get_exact_count(h, stream: int, clear: bool = True) -> int:
+    n = ctypes.c_uint32()
+    check(lib().sq_get_exact_count(h, stream, ctypes.byref(n), 1 if clear else 0))
+    return n.value
+
+
+def sq_launch_plan(h) -> dict:
+    v = [ctypes.c_int32() for _ in range(5)]
+    check(lib().sq_launch_plan(h, *[ctypes.byref(x) for x in v]))
+    return dict(zip(("grid", "threads", "ctas_per_sm", "stages", "smem_bytes"), (x.value for x in v)))
+
+
+def sq_set_wait_limit(h, ns: int) -> None:
+    check(lib().sq_set_wait_limit(h, int(ns)))
+
+
+def sq_test_stall_stages(h, extra_bytes: int) -> None:
+    check(lib().sq_test_stall_stages(h, int(extra_bytes)))
 
 
 def sq_decode_step_noalloc(desc: StateDesc, calib: Calib, pool, q, k, v, beta, g, o, slot_ids, B, status,

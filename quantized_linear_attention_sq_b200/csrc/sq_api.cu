@@ -14,6 +14,7 @@
 #include "sq_host.h"
 #include "sq_kernels.cuh"
 #include "sq_prefill.cuh"
+#include "sq_step.cuh"
 
 namespace sqi {
 
@@ -63,6 +64,9 @@ inline float clip_ratio(float phi) { return phi < 1.0f ? phi : 1.0f; }
 // unchanged).
 constexpr int kStepChunk = 1;
 
+// Limit of the kernels' bounded waits (a stage's data, the partials buffer).
+constexpr uint64_t kWaitNs = 2000000000ull;
+
 }  // namespace
 
 struct sq_handle {
@@ -85,6 +89,8 @@ struct sq_handle {
   uint64_t stage_rec = 0;  // largest record that goes through a stage
   size_t step_smem = 0;
   uint64_t launches = 0;
+  uint64_t wait_ns = kWaitNs;     // limit of the kernels' bounded waits
+  uint32_t test_extra_tx = 0;     // testing only (sq_test_stall_stage)
   // sq_decode_step_host: two device staging sets used in turn, the internal
   // stream their host-to-device copies run on, and the events that order
   // the copies after the step that last read a set.
@@ -101,14 +107,27 @@ struct sq_handle {
 
 namespace {
 
-template <int D>
-constexpr int threads_for() { return sqk::Geo<D>::NT; }
-
+// Threads per CTA of the FP32 step, quantize and dequantize (Geo) and of
+// the packed step (PGeo).
 int threads_of(int d) {
   switch (d) {
-    case 128: return threads_for<128>();
-    case 64: return threads_for<64>();
-    default: return threads_for<32>();
+    case 128: return sqk::Geo<128>::NT;
+    case 64: return sqk::Geo<64>::NT;
+    default: return sqk::Geo<32>::NT;
+  }
+}
+int packed_threads_of(int d) {
+  switch (d) {
+    case 128: return sqk::PGeo<128>::NT;
+    case 64: return sqk::PGeo<64>::NT;
+    default: return sqk::PGeo<32>::NT;
+  }
+}
+uint32_t packed_aux_of(int d) {
+  switch (d) {
+    case 128: return sqk::PGeo<128>::AUX;
+    case 64: return sqk::PGeo<64>::AUX;
+    default: return sqk::PGeo<32>::AUX;
   }
 }
 
@@ -120,8 +139,11 @@ cudaError_t allow_max_smem(K kernel, int max_smem) {
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              max_smem - (int)fa.sharedSizeBytes);
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem - (int)fa.sharedSizeBytes);
+  if (e != cudaSuccess) return e;
+  // all of the unified L1 / shared storage as shared memory, so that as
+  // many CTAs fit per SM as the occupancy calculation assumes
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
 }
 
 template <int D>
@@ -156,11 +178,11 @@ struct StepPlan {
 };
 
 // Packed pools: a stage holds one record (every head except the all-pivot
-// ones, which the kernel reads in place) plus the tile's vectors; the S^T k
-// and o partials share one buffer of 32 d fp64 values. The pipeline needs
-// at least 2 stages. Preference: as many CTAs per SM as registers allow (at
-// most 3, with 2 stages), then as many stages as fit (at most 4). FP32
-// pools: 1 CTA per SM, up to 4 stages.
+// ones, which the kernel reads in place) plus the tile's vectors and row
+// tables; the S^T k (fp64) and o partials share one buffer of 16 d fp64
+// values. Two stages; as many CTAs per SM as registers and shared memory
+// allow (at most 4 at d = 128). FP32 pools: 1 CTA per SM, up to 4 stages
+// (the FP32 kernel's partials buffer is 32 d fp32 values).
 sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int optin_smem, int reserved_smem,
                       StepPlan* p) {
   const void* kern = step_kernel_of(d, packed);
@@ -168,33 +190,33 @@ sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int o
   cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
   const size_t static_smem = fa.sharedSizeBytes;
+  const int nt = packed ? packed_threads_of(d) : threads_of(d);
   p->rec_cap = (uint32_t)round_up(stage_rec < 16 ? 16 : stage_rec, 128);
-  p->stage_bytes = (uint32_t)round_up(p->rec_cap + 32u * d + 32u, 128);  // + vectors, tables, header
-  const int NG = 32;  // row groups per CTA: 32 for every supported d
-  const size_t red = (size_t)NG * d * (packed ? 8 : 4);
+  p->stage_bytes = packed ? (uint32_t)round_up(p->rec_cap + packed_aux_of(d), 128)
+                          : (uint32_t)round_up(p->rec_cap + 32u * d + 32u, 128);
+  const size_t red = packed ? (size_t)16 * d * 8 : (size_t)32 * d * 4;
   const size_t dyn_max = (size_t)optin_smem - static_smem;
-  const int min_ns = packed ? 2 : 1;
-  // CTAs per SM allowed by registers and threads alone
   int by_regs = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&by_regs, kern, threads_of(d), 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&by_regs, kern, nt, 0);
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
-  int first = packed ? 3 : 1;
-  if (by_regs >= 1 && by_regs < first) first = by_regs;
+  if (by_regs < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
   p->nstage = 0;
-  for (int want = first; want >= 1 && p->nstage == 0; --want) {
-    const long budget = (long)sm_smem / want - reserved_smem - (long)static_smem;
-    if (budget < (long)red) continue;
-    int ns = (int)((size_t)(budget - (long)red) / p->stage_bytes);
-    if (ns > 4) ns = 4;
-    if (want == 3 && ns > 2) ns = 2;
-    if (ns < min_ns) continue;
+  if (packed) {
+    const int ns = 2;
     const size_t smem = (size_t)ns * p->stage_bytes + red;
-    if (smem > dyn_max) continue;
+    if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
     p->nstage = ns;
     p->smem = smem;
+  } else {
+    const long budget = (long)sm_smem - reserved_smem - (long)static_smem;
+    int ns = budget > (long)red ? (int)((size_t)(budget - (long)red) / p->stage_bytes) : 0;
+    if (ns > 4) ns = 4;
+    if (ns < 1) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
+    p->nstage = ns;
+    p->smem = (size_t)ns * p->stage_bytes + red;
+    if (p->smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
   }
-  if (p->nstage == 0) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p->blocks, kern, threads_of(d), p->smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p->blocks, kern, nt, p->smem);
   if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
   if (p->blocks < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
   return SQ_OK;
@@ -279,12 +301,14 @@ sq_status launch_step(sq_handle* h, void* pool, const float* q, const float* k, 
   a.nstage = h->nstage; a.rec_cap = h->rec_cap; a.stage_bytes = h->stage_bytes;
   a.chunk = kStepChunk;
   a.slot_bytes = h->slot_bytes;
+  a.wait_ns = h->wait_ns;
+  a.test_extra_tx = h->test_extra_tx;
   a.t = h->tables;
   const int n_tiles = B * h->desc.h_v;
   const int grid = n_tiles < h->step_grid ? n_tiles : h->step_grid;
-  const int nt = threads_of(h->d);
-  cudaStream_t st = as_stream(stream);
   const bool packed = h->desc.fmt == SQ_FMT_PACKED;
+  const int nt = packed ? packed_threads_of(h->d) : threads_of(h->d);
+  cudaStream_t st = as_stream(stream);
   if (packed) {
     if (h->d == 128) sqk::k_decode_step_packed<128><<<grid, nt, h->step_smem, st>>>(a);
     else if (h->d == 64) sqk::k_decode_step_packed<64><<<grid, nt, h->step_smem, st>>>(a);
@@ -439,6 +463,7 @@ sq_status sq_state_alloc(const sq_state_desc* desc, const sq_calib* calib, void*
   h->tables.row_perm = reinterpret_cast<const uint8_t*>(base + o_row_perm);
   h->tables.head_kind = reinterpret_cast<const uint8_t*>(base + o_head_kind);
   h->tables.status = reinterpret_cast<uint32_t*>(base + o_status);
+  h->tables.xcount = reinterpret_cast<uint32_t*>(base + o_status + 4);
   h->tables.sched = reinterpret_cast<uint32_t*>(base + o_status + 8);  // zero, and reset by every step launch
   s = plan_step(h);
   if (s != SQ_OK) {
@@ -492,6 +517,47 @@ sq_status sq_head_layout(const sq_handle* h, int32_t head, uint64_t* offset, uin
 }
 
 uint64_t sq_launch_count(const sq_handle* h) { return h ? h->launches : 0; }
+
+sq_status sq_get_exact_count(sq_handle* h, void* stream, uint32_t* count, int32_t clear) {
+  g_last_error.clear();
+  if (!h || !count) return fail(SQ_ERR_INVALID_ARG, "NULL argument");
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, h->tables.xcount, 4, cudaMemcpyDeviceToHost, as_stream(stream));
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(h->tables.xcount, 0, 4, as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the exact-sum count");
+  *count = v;
+  return SQ_OK;
+}
+
+sq_status sq_launch_plan(const sq_handle* h, int32_t* grid, int32_t* threads, int32_t* ctas_per_sm,
+                         int32_t* stages, int32_t* smem_bytes) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  const bool packed = h->desc.fmt == SQ_FMT_PACKED;
+  if (grid) *grid = h->step_grid;
+  if (threads) *threads = packed ? packed_threads_of(h->d) : threads_of(h->d);
+  if (ctas_per_sm) *ctas_per_sm = h->num_sms ? h->step_grid / h->num_sms : 0;
+  if (stages) *stages = h->nstage;
+  if (smem_bytes) *smem_bytes = (int32_t)h->step_smem;
+  return SQ_OK;
+}
+
+sq_status sq_set_wait_limit(sq_handle* h, uint64_t ns) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (ns < 1000) return fail(SQ_ERR_INVALID_ARG, "wait limit %llu ns is below 1000", (unsigned long long)ns);
+  h->wait_ns = ns;
+  return SQ_OK;
+}
+
+sq_status sq_test_stall_stages(sq_handle* h, uint32_t extra_bytes) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (extra_bytes > 65536u) return fail(SQ_ERR_INVALID_ARG, "extra_bytes %u above 65536", extra_bytes);
+  h->test_extra_tx = extra_bytes;
+  return SQ_OK;
+}
 
 sq_status sq_get_status(sq_handle* h, void* stream, uint32_t* bits, int32_t clear) {
   g_last_error.clear();
@@ -912,6 +978,8 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.slots = slot_ids;
   a.B = B; a.h_v = hv; a.h_k = desc->h_k; a.n_slots = desc->n_slots; a.gate_kind = desc->gate;
   a.slot_bytes = off;
+  a.wait_ns = kWaitNs;
+  a.test_extra_tx = 0;
   a.t.rec_off = reinterpret_cast<const uint32_t*>(nd->scratch + o_rec_off);
   a.t.rec_bytes = reinterpret_cast<const uint32_t*>(nd->scratch + o_rec_bytes);
   a.t.col = reinterpret_cast<const float*>(nd->scratch + o_col);
@@ -922,6 +990,7 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
   a.t.row_perm = reinterpret_cast<const uint8_t*>(nd->scratch + o_row_perm);
   a.t.head_kind = reinterpret_cast<const uint8_t*>(nd->scratch + o_head_kind);
   a.t.status = status ? status : reinterpret_cast<uint32_t*>(nd->scratch + o_status);
+  a.t.xcount = reinterpret_cast<uint32_t*>(nd->scratch + o_status + 4);
   a.t.sched = reinterpret_cast<uint32_t*>(nd->scratch + o_status + 8);  // uploaded as zeros above
 
   // launch plan (same rule as a handle's)
@@ -941,9 +1010,9 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
     e = cudaMemsetAsync(nd->scratch + o_status, 0, 4, st);  // the scratch status word starts at zero
     if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch status word");
   }
-  if (d == 128) sqk::k_decode_step_packed<128><<<grid, threads_of(128), smem, st>>>(a);
-  else if (d == 64) sqk::k_decode_step_packed<64><<<grid, threads_of(64), smem, st>>>(a);
-  else sqk::k_decode_step_packed<32><<<grid, threads_of(32), smem, st>>>(a);
+  if (d == 128) sqk::k_decode_step_packed<128><<<grid, packed_threads_of(128), smem, st>>>(a);
+  else if (d == 64) sqk::k_decode_step_packed<64><<<grid, packed_threads_of(64), smem, st>>>(a);
+  else sqk::k_decode_step_packed<32><<<grid, packed_threads_of(32), smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching the no-alloc decode step");
   return SQ_OK;

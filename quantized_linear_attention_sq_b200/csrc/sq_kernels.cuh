@@ -1,28 +1,23 @@
-// sq_kernels.cuh -- sm_100a kernels of the quantized-state decode step.
+// sq_kernels.cuh -- sm_100a building blocks of the quantized-state decode
+// step, and the kernels around it.
 //
-// One CTA owns one (request, value head) state tile at a time. CTAs are
-// persistent and take tiles in turn (the packed step claims them from a work
-// counter); the records (plus the tile's small vectors and head tables) arrive in shared
-// memory through 1-D TMA bulk copies (cp.async.bulk, no multicast) completed
-// on an mbarrier, NSTAGE tiles ahead of the one being computed. The updated
-// record is written back in place from shared memory with a bulk store. The
-// state therefore crosses HBM exactly once in each direction per step
-// ("STEPQuant: estados recurrentes a 6 bit" (gpt-diffusion), section "Las
-// dos ideas": fused kernels that move the packed state, not FP32).
+// The FP32-state baseline step is persistent like the packed step: one CTA
+// owns one (request, value head) tile at a time, the tile (plus its small
+// vectors) arrives in shared memory through 1-D TMA bulk copies
+// (cp.async.bulk, no multicast) completed on an mbarrier, NSTAGE tiles ahead
+// of the one being computed, and goes back in place with a bulk store.
+// Thread map of the kernels in this file (Geo): a thread owns 16
+// consecutive value columns of RPT key rows (d = 128: 256 threads, 4 rows
+// each; 8 lanes cover one row, so a row's 16-column chunk is 2*b bytes =
+// b/2 whole 32-bit words for every width b). Column sums go through shared
+// memory; row maxima use warp shuffles over the lanes of a row.
 //
-// Thread map for a d x d tile: a thread owns 16 consecutive value columns of
-// RPT key rows (d = 128: 256 threads, 4 rows each; 8 lanes cover one row, so
-// a row's 16-column chunk is 2*b bytes = b/2 whole 32-bit words for every
-// width b). Column sums (S^T k, S^T q) go through shared memory; row maxima
-// use warp shuffles over the 8 lanes of a row.
-//
-// Arithmetic follows a fixed elementwise recipe so that codes are
-// reproducible: a_i = r_i g_i; T = q a_i; P_j = sum_i T_ij k_i;
-// u_j = beta (v_j - c_j P_j); w_j = u_j / c_j (as u_j * fl(1/c_j));
-// T' = fma(k_i, w_j, T); o_j = c_j sum_i T'_ij q_i; m_i = max_j |T'_ij|;
-// r'_i = fp16 round-up of (phi_i m_i) / qmax; q' = RNE(clamp(T' * fl(1/r'))),
-// with phi_i the clip ratio from the tables.
-// Only the two column sums depend on summation order.
+// The fused packed step itself is in sq_step.cuh; this file holds the code
+// formats (bit-field unpacking and packing, fp16 pivots), the shared
+// requantization helpers, the FP32-state baseline step and the quantize /
+// dequantize kernels. Every elementwise operation is an explicit
+// round-to-nearest intrinsic (the library is built with --fmad=false), so
+// codes are reproducible.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -51,6 +46,7 @@ struct Tables {
   const uint8_t* head_kind;   // [h_v] width shared by all rows of the head (ROW_PIVOT: all pivot), 0: mixed
   uint32_t* status;           // device status word
   uint32_t* sched;            // packed step: [0] next chunk of tiles, [1] CTAs done (both 0 between launches)
+  uint32_t* xcount;           // packed step: columns whose S^T k was summed exactly (running count)
 };
 
 struct StepArgs {
@@ -68,6 +64,8 @@ struct StepArgs {
   uint32_t rec_cap;     // bytes reserved for a record in a stage (multiple of 128)
   uint32_t stage_bytes; // rec_cap + aux bytes, multiple of 128
   uint64_t slot_bytes;
+  uint64_t wait_ns;     // limit of every bounded wait inside the kernel
+  uint32_t test_extra_tx;  // testing only: extra bytes CTA 0 expects per stage (0: none)
   Tables t;
 };
 
@@ -295,33 +293,6 @@ __device__ __forceinline__ void chunk_words(const uint8_t* row, int cc, uint32_t
   } else {
 #pragma unroll
     for (int i = 0; i < B / 2; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
-  }
-}
-
-// High words of the fp64 views of the 8 values of half H of a chunk, and
-// the same 8 values as floats (codes q, or fp16 pivot values).
-template <int B, int H>
-__device__ __forceinline__ void hi_half_q(const uint32_t (&w)[B / 2], uint32_t (&xh)[8], float2 (&V)[4]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) xh[j] = field_hi<B>(w, 8 * H + j);
-  // scalar fmas: each value lands directly in its pair register (an f32x2
-  // fma would need xh[2p], xh[2p+1] in an aligned pair, which the fp64 views
-  // of the same words also claim)
-  constexpr float K = FieldPos<B>::K, C = FieldPos<B>::C;
-#pragma unroll
-  for (int p = 0; p < 4; ++p)
-    V[p] = make_float2(__fmaf_rn(__uint_as_float(xh[2 * p]), K, -C), __fmaf_rn(__uint_as_float(xh[2 * p + 1]), K, -C));
-}
-// Pivot chunk: the fp16 values themselves (an fp16 value as a double has a
-// zero low word).
-template <int H>
-__device__ __forceinline__ void hi_half_pivot(const uint32_t (&w)[8], uint32_t (&xh)[8], float2 (&V)[4]) {
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[4 * H + p]));
-    V[p] = x;
-    xh[2 * p] = (uint32_t)__double2hiint((double)x.x);
-    xh[2 * p + 1] = (uint32_t)__double2hiint((double)x.y);
   }
 }
 
@@ -877,20 +848,10 @@ __global__ void __launch_bounds__(Geo<D>::NT, 1) k_decode_step_fp32(const StepAr
 }
 
 // ----------------------------------------------------------- packed state
-// Per tile, three block barriers:
-//   wait for the stage; pass A: codes -> fp64 column partials of S^T k
-//   B1; column totals -> P, w = beta (v - c P) / c
-//   B2; pass B: codes read again -> T' = q a + k w (one rounding), o
-//       partials, row maxima, row scales, new codes written in place
-//   B3; o = c (column totals); thread 0 stores the record, and refills
-//       the stage right after the next tile's B1.
-// The partials of S^T k (fp64) and of S'^T q (fp32) share one buffer: a
-// thread deposits the next tile's S^T k partials only after every thread
-// has read this tile's o partials (an mbarrier every thread arrives on).
-
-// Tiles are numbered head-major, m = h B + b, and handed out in chunks of
-// a.chunk consecutive tiles from a global counter: a CTA works on one head
-// (one width, one code path) for several tiles in a row, and the CTAs stay
+// Scheduling helpers of the persistent packed step (sq_step.cuh). Tiles are
+// numbered head-major, m = h B + b, and handed out in chunks of a.chunk
+// consecutive tiles from a global counter: a CTA works on one head (one
+// width, one code path) for several tiles in a row, and the CTAs stay
 // balanced although the widths cost differently.
 //
 // Control block of the producing thread (shared memory, thread 0 only).
@@ -956,534 +917,11 @@ __device__ __forceinline__ void producer_start(const StepArgs& a, Producer* pr, 
   prefetch_scalars(a, pr, pr->next, 0);
 }
 
-// Issue tile x into a stage. All-pivot heads (kind ROW_PIVOT) are not
-// staged: their fp16 record is read and written in place in the pool, with
-// the L2 warmed by a bulk prefetch, so stages are sized for the largest
-// other record.
-template <int D>
-__device__ __forceinline__ void issue_packed(const StepArgs& a, const TileScalars& x, uint8_t* stage_base,
-                                             uint64_t* bar) {
-  Stage<D> s{stage_base, a.rec_cap};
-  TileHdr* hd = s.hdr();
-  hd->tile = x.b * a.h_v + x.h;
-  if (x.slot < 0 || x.slot >= a.n_slots) {
-    hd->valid = 0;
-    mbar_arrive(bar);
-    return;
-  }
-  const int b = x.b, h = x.h;
-  const int hk = h / (a.h_v / a.h_k);
-  const uint32_t vec = 4u * D;
-  const bool kda = a.gate_kind != 0;
-  const bool direct = x.kind == ROW_PIVOT;
-  uint8_t* rec_src = a.pool + (uint64_t)x.slot * a.slot_bytes + x.rec_off;
-  hd->dst = rec_src;
-  hd->bytes = x.rec_bytes;
-  hd->valid = 1;
-  hd->beta = x.beta;
-  hd->g = x.g;
-  hd->kind = x.kind;
-  const bool mixed = x.kind == 0;  // rows of different widths: the row order is needed
-  uint32_t tx = 6u * vec + (kda ? vec : 0u) + 3u * D + (mixed ? (uint32_t)D : 0u);
-  if (!direct) tx += x.rec_bytes;
-  mbar_arrive_expect_tx(bar, tx);
-  if (direct)
-    bulk_prefetch_l2(rec_src, x.rec_bytes);
-  else
-    bulk_g2s(s.rec(), rec_src, x.rec_bytes, bar);
-  bulk_g2s(s.k(), a.k + ((size_t)b * a.h_k + hk) * D, vec, bar);
-  bulk_g2s(s.q(), a.q + ((size_t)b * a.h_k + hk) * D, vec, bar);
-  bulk_g2s(s.v(), a.v + ((size_t)b * a.h_v + h) * D, vec, bar);
-  if (kda) bulk_g2s(s.g(), a.g + ((size_t)b * a.h_v + h) * D, vec, bar);
-  bulk_g2s(s.c(), a.t.col + (size_t)h * D, vec, bar);
-  bulk_g2s(s.ic(), a.t.icol + (size_t)h * D, vec, bar);
-  bulk_g2s(s.phi(), a.t.phi + (size_t)h * D, vec, bar);
-  bulk_g2s(s.row_off(), a.t.row_off + (size_t)h * D, 2u * D, bar);
-  bulk_g2s(s.row_code(), a.t.row_code + (size_t)h * D, (uint32_t)D, bar);
-  if (mixed) bulk_g2s(s.row_perm(), a.t.row_perm + (size_t)h * D, (uint32_t)D, bar);
-}
-
-// Thread 0: issue the next tile into stage s (or mark the stage as the end
-// of the work), then start fetching the scalars of the tile after it,
-// claiming a new chunk when the current one is used up.
-template <int D>
-__device__ __forceinline__ void issue_next(const StepArgs& a, Producer* pr, uint8_t* stages, uint64_t* bars, int s,
-                                           int& ahead) {
-  uint8_t* base = stages + (size_t)s * a.stage_bytes;
-  const int m = pr->next;
-  if (m < 0) {
-    Stage<D>{base, a.rec_cap}.hdr()->tile = -1;
-    return;
-  }
-  cp_async_wait_all();
-  const int k = pr->buf;
-  TileScalars x;
-  x.h = m / a.B;
-  x.b = m - x.h * a.B;
-  x.tile = x.b * a.h_v + x.h;
-  x.slot = pr->slot[k];
-  x.rec_off = pr->rec_off[k];
-  x.rec_bytes = pr->rec_bytes[k];
-  x.kind = (int)((pr->kind_word[k] >> (8 * (x.h & 3))) & 0xFFu);
-  x.beta = pr->beta[k];
-  x.g = a.gate_kind == 0 ? pr->g[k] : 0.0f;
-  int nm = m + 1;
-  if (nm >= pr->end) {
-    const int n_tiles = a.B * a.h_v;
-    const int n_chunks = (n_tiles + a.chunk - 1) / a.chunk;
-    const int c = ahead;  // claimed a chunk ago
-    if (c < n_chunks) {
-      nm = c * a.chunk;
-      pr->end = min(nm + a.chunk, n_tiles);
-      ahead = (int)atomicAdd(a.t.sched, 1u);
-    } else {
-      nm = -1;
-    }
-  }
-  pr->next = nm;
-  pr->buf = k ^ 1;
-  prefetch_scalars(a, pr, nm, k ^ 1);
-  issue_packed<D>(a, x, base, &bars[s]);
-}
-
-// Thread 0: refill the stage whose store is pending, once the store has
-// read it (tiles go to stages round-robin, so the next tile to issue is
-// the one that belongs to that stage).
-template <int D>
-__device__ __forceinline__ void refill_pending(const StepArgs& a, Producer* pr, uint8_t* stages, uint64_t* bars,
-                                               int& ahead) {
-  const int s = pr->pend;
-  if (s < 0) return;
-  pr->pend = -1;
-  bulk_wait_read_all();
-  issue_next<D>(a, pr, stages, bars, s, ahead);
-}
-
-// Pass A, half H (8 columns) of a thread's chunk over its rows, for a head
-// of uniform width B (B = 16: all-pivot head, read from the pool when
-// DIRECT): the values go to T[r][4H..4H+3], the fp64 partials of S^T k to
-// acc. Only the words of half H are loaded.
-template <int D, int B, int H, bool DIRECT>
-__device__ __forceinline__ void pass_a_half(const uint8_t* rec, int rg, int cc, const double (&kap)[Geo<D>::RPT],
-                                            double acc0, float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
-  uint32_t w[Geo<D>::RPT][B / 2];
-#pragma unroll
-  for (int r = 0; r < Geo<D>::RPT; ++r)
-    chunk_words<B, DIRECT>(rec + row_offset<D, B>(nullptr, r * Geo<D>::NG + rg), cc, w[r]);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = acc0;
-#pragma unroll
-  for (int r = 0; r < Geo<D>::RPT; ++r) {
-    uint32_t xh[8];
-    float2 V[4];
-    if constexpr (B == 16)
-      hi_half_pivot<H>(w[r], xh, V);
-    else
-      hi_half_q<B, H>(w[r], xh, V);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) T[r][4 * H + p] = V[p];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap[r], acc[j]);
-  }
-}
-
-// Same for a head whose rows have different widths (one unit per key row).
-// The row's width decides the unpacking; values pass through temporaries
-// (writing T[r] inside the switch would send the tile to local memory).
-// Row offsets are clamped to the stage's record capacity: every read then
-// stays inside the stage even if its tables were never loaded (a wait that
-// gave up).
-template <int D, int H>
-__device__ __forceinline__ void pass_a_half_mixed(const uint8_t* rec, const uint16_t* row_off,
-                                                  const uint8_t* row_code, const uint8_t* row_perm,
-                                                  uint32_t rec_cap, int rg, int cc,
-                                                  const double (&kap)[Geo<D>::RPT], double acc0,
-                                                  float2 (&T)[Geo<D>::RPT][8], double (&acc)[8]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = acc0;
-#pragma unroll
-  for (int r = 0; r < Geo<D>::RPT; ++r) {
-    const int i = row_perm[r * Geo<D>::NG + rg] & (D - 1);  // (masked: in bounds even if never loaded)
-    const uint8_t* row = rec + min((uint32_t)row_off[i], rec_cap);
-    uint32_t xh[8];
-    float2 V[4];
-    switch (row_code[i]) {
-      case 8: { uint32_t w[4]; chunk_words<8, false, false>(row, cc, w); hi_half_q<8, H>(w, xh, V); } break;
-      case 6: { uint32_t w[3]; chunk_words<6, false, false>(row, cc, w); hi_half_q<6, H>(w, xh, V); } break;
-      case 4: { uint32_t w[2]; chunk_words<4, false, false>(row, cc, w); hi_half_q<4, H>(w, xh, V); } break;
-      case 2: { uint32_t w[1]; chunk_words<2, false, false>(row, cc, w); hi_half_q<2, H>(w, xh, V); } break;
-      default: { uint32_t w[8]; chunk_words<16, false, false>(row, cc, w); hi_half_pivot<H>(w, xh, V); } break;
-    }
-#pragma unroll
-    for (int p = 0; p < 4; ++p) T[r][4 * H + p] = V[p];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = fma(__hiloint2double((int)xh[j], 0), kap[r], acc[j]);
-  }
-}
-
 // max(|a|, |b|, |c|), NaN if any input is NaN (one instruction on sm_100).
 __device__ __forceinline__ float absmax3_nan(float a, float b, float c) {
   float r;
   asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// max_j |T'_j| over the 16 values of a chunk (a depth-3 tree), then over
-// the LPR lanes of the row; NaN if any value of the row is NaN.
-template <int D>
-__device__ __forceinline__ float row_absmax(const float2 (&t)[8]) {
-  const float a0 = absmax3_nan(t[0].x, t[0].y, t[1].x);
-  const float a1 = absmax3_nan(t[1].y, t[2].x, t[2].y);
-  const float a2 = absmax3_nan(t[3].x, t[3].y, t[4].x);
-  const float a3 = absmax3_nan(t[4].y, t[5].x, t[5].y);
-  const float a4 = absmax3_nan(t[6].x, t[6].y, t[7].x);
-  const float b0 = absmax3_nan(a0, a1, a2);
-  const float b1 = absmax3_nan(a3, a4, t[7].y);
-  float x = fmax_nan(b0, b1);
-#pragma unroll
-  for (int s = 1; s < Geo<D>::LPR; s <<= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, s));
-  return x;
-}
-
-// Requantization of RB rows (group grp of a thread's row slots): row maxima
-// over the LPR lanes of each row, one row scale per row (lane cc % RB of
-// the row group computes it, the others take it by shuffle), codes. Writes
-// the record (shared memory, or the pool for an all-pivot head). Pivot rows
-// keep their scale slot. A row holding a NaN gets scale 0 and all codes 0;
-// such rows are found with one warp vote, so the common case runs without
-// per-row tests.
-template <int D, int KC, int RB>
-__device__ __forceinline__ uint32_t requant_group(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
-                                                  const uint8_t* row_perm, const float* phi, int grp, int rg,
-                                                  int cc, const float2 (&T)[RB][8]) {
-  using G = Geo<D>;
-  uint32_t st = 0;
-  if constexpr (KC == ROW_PIVOT) {
-#pragma unroll
-    for (int u = 0; u < RB; ++u)
-      st |= store_row_pivot<true>(rec + row_offset<D, KC>(row_off, (grp * RB + u) * G::NG + rg), cc, T[u]);
-    return st;
-  } else {
-    float m[RB];
-    bool nan_row = false;
-#pragma unroll
-    for (int u = 0; u < RB; ++u) {
-      m[u] = row_absmax<D>(T[u]);
-      nan_row |= m[u] != m[u];
-    }
-    const int mine = cc % RB;
-    float mm = m[0];
-#pragma unroll
-    for (int u = 1; u < RB; ++u) mm = mine == u ? m[u] : mm;
-    const int sm = (grp * RB + mine) * G::NG + rg;  // slot
-    const int im = KC ? sm : row_perm[sm];           // row
-    const int cm = KC ? KC : row_code[im];
-    float ir_m = 0.0f, lim_m = 0.0f;
-    if (cm != ROW_PIVOT) {
-      uint16_t rbits = 0;
-      if (mm == mm) {
-        const float qm = (float)((1 << (cm - 1)) - 1);
-        const float s = __fdiv_rn(__fmul_rn(phi[im], mm), qm);
-        __half rh;
-        if (s > 65504.0f) {
-          rh = __ushort_as_half((unsigned short)0x7BFF);
-          st |= ST_SAT;
-        } else {
-          rh = __float2half_ru(s);
-        }
-        const float R = __half2float(rh);
-        ir_m = (R == 0.0f) ? 0.0f : __frcp_rn(R);
-        lim_m = __fmul_rn(qm, R);  // qmax r', exact
-        rbits = __half_as_ushort(rh);
-      }
-      if (cc < RB) reinterpret_cast<uint16_t*>(rec)[im] = rbits;
-    }
-    const int base = (int)(threadIdx.x & 31) - cc;
-    if (!__any_sync(0xffffffffu, nan_row)) {
-#pragma unroll
-      for (int u = 0; u < RB; ++u) {
-        const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
-        const float lim = __shfl_sync(0xffffffffu, lim_m, base + u);
-        const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
-        const int code = KC ? KC : row_code[i];
-        uint8_t* row = rec + row_offset<D, KC>(row_off, i);
-        switch (code) {
-          case 8: store_row_q<8>(row, cc, ir, lim, T[u]); break;
-          case 6: store_row_q<6>(row, cc, ir, lim, T[u]); break;
-          case 4: store_row_q<4>(row, cc, ir, lim, T[u]); break;
-          case 2: store_row_q<2>(row, cc, ir, lim, T[u]); break;
-          default: st |= store_row_pivot<false>(row, cc, T[u]); break;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < RB; ++u) {
-        const float ir = __shfl_sync(0xffffffffu, ir_m, base + u);
-        const float lim = __shfl_sync(0xffffffffu, lim_m, base + u);
-        const int i = KC ? (grp * RB + u) * G::NG + rg : row_perm[(grp * RB + u) * G::NG + rg];
-        const int code = KC ? KC : row_code[i];
-        uint8_t* row = rec + row_offset<D, KC>(row_off, i);
-        if (code == ROW_PIVOT) {
-          st |= store_row_pivot<false>(row, cc, T[u]);
-        } else if (m[u] != m[u]) {
-          st |= ST_NAN;
-          store_row_zero(row, code, cc);
-        } else {
-          switch (code) {
-            case 8: store_row_q<8>(row, cc, ir, lim, T[u]); break;
-            case 6: store_row_q<6>(row, cc, ir, lim, T[u]); break;
-            case 4: store_row_q<4>(row, cc, ir, lim, T[u]); break;
-            default: store_row_q<2>(row, cc, ir, lim, T[u]); break;
-          }
-        }
-      }
-    }
-    return st;
-  }
-}
-
-// One tile of the packed step. KC is the width shared by every row of the
-// head (ROW_PIVOT: an all-pivot head, whose record stays in the pool), or 0
-// for heads whose rows differ; with KC != 0 every per-row width test folds
-// away. Returns false when a bounded wait gave up (the tile is abandoned).
-template <int D, int KC>
-__device__ __forceinline__ bool packed_tile(const StepArgs& a, const Stage<D>& S, int sidx, uint32_t parity, int n,
-                                            uint64_t* bars, uint64_t* free_bar, uint8_t* stages, uint8_t* red,
-                                            float* wsh, float* msh, int* abort_sh, Producer* pr,
-                                            int& ahead, float* o, int rg, int cc, uint32_t& st) {
-  using G = Geo<D>;
-  constexpr bool DIRECT = KC == ROW_PIVOT;
-  const int tid = threadIdx.x;
-  const int base = (tid & 31) - cc;
-  const bool kda = a.gate_kind != 0;
-  const TileHdr* hd = S.hdr();
-  uint8_t* rec = DIRECT ? hd->dst : S.rec();
-  double* red64 = reinterpret_cast<double*>(red);
-
-  // ---- pass A: the tile's values into registers (T), fp64 column
-  // partials of S^T k
-  // A thread whose wait gave up still runs pass A, on stale but in-bounds
-  // shared memory, and the tile is abandoned at B1 before anything is
-  // written (keeping pass A unconditional keeps the tile in registers).
-  float2 T[G::RPT][8];
-  if (!mbar_wait_bounded(&bars[sidx], parity, 2000000000ull)) *abort_sh = 1;
-  {
-    // row factors: lane cc computes row slot cc % RPT, the others take it
-    // by shuffle. M = fp32(r g) (quantized row) or g (pivot row); the fp64
-    // weight kap = M k is exact.
-    const int mine = cc % G::RPT;
-    const int sm = mine * G::NG + rg;                  // slot
-    const int im = KC ? sm : (S.row_perm()[sm] & (D - 1));  // row (masked: in bounds even if never loaded)
-    const int cm = KC ? KC : S.row_code()[im];
-    const float gm = kda ? S.g()[im] : hd->g;
-    const float mm =
-        cm == ROW_PIVOT ? gm : __fmul_rn(__half2float(reinterpret_cast<const __half*>(rec)[im]), gm);
-    if (cc < G::RPT) msh[sm] = mm;
-    const double kapm = (double)mm * (double)S.k()[im];
-    double kap[G::RPT];
-    double off = 0.0;
-#pragma unroll
-    for (int r = 0; r < G::RPT; ++r) {
-      kap[r] = __shfl_sync(0xffffffffu, kapm, base + r);
-      const int code = KC ? KC : S.row_code()[S.row_perm()[r * G::NG + rg] & (D - 1)];
-      if (code != ROW_PIVOT) off = fma(code_offset(code), kap[r], off);
-    }
-    bool free_ok = true;
-    double acc[8];
-    // the accumulators start at -off, the rows' bias (see code_offset)
-    if constexpr (KC != 0) {
-      pass_a_half<D, KC, 0, DIRECT>(rec, rg, cc, kap, -off, T, acc);
-      // the buffer is free once every thread has read the previous tile's o partials
-      if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc);
-      pass_a_half<D, KC, 1, DIRECT>(rec, rg, cc, kap, -off, T, acc);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc);
-    } else {
-      pass_a_half_mixed<D, 0>(rec, S.row_off(), S.row_code(), S.row_perm(), a.rec_cap, rg, cc, kap, -off, T,
-                              acc);
-      if (n > 0) free_ok = mbar_wait_bounded(free_bar, (uint32_t)(n - 1) & 1u, 2000000000ull);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 0, acc);
-      pass_a_half_mixed<D, 1>(rec, S.row_off(), S.row_code(), S.row_perm(), a.rec_cap, rg, cc, kap, -off, T,
-                              acc);
-      if (free_ok) deposit_f64<D>(red64, rg, cc, 1, acc);
-    }
-    if (!free_ok) *abort_sh = 1;
-  }
-  __syncthreads();  // B1: the S^T k partials are complete
-  if (*abort_sh) return false;
-  if (tid == 0) refill_pending<D>(a, pr, stages, bars, ahead);
-
-  // ---- column totals of S^T k -> w
-  {
-    const float P = column_total_f64<D>(red64);
-    if ((tid & 1) == 0) {
-      const int j = tid >> 1;
-      const float p = __fmul_rn(S.c()[j], P);
-      const float u = __fmul_rn(hd->beta, __fsub_rn(S.v()[j], p));
-      wsh[j] = __fmul_rn(u, S.ic()[j]);
-    }
-  }
-  __syncthreads();  // B2: w is complete
-
-  // ---- pass B: update (one rounding), o partials, requantization
-  float2 W[8];
-  {
-    const float4* wsrc = reinterpret_cast<const float4*>(wsh + 16 * cc);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float4 x = wsrc[p];
-      W[2 * p] = make_float2(x.x, x.y);
-      W[2 * p + 1] = make_float2(x.z, x.w);
-    }
-  }
-  float2 part[8];
-#pragma unroll
-  for (int r = 0; r < G::RPT; ++r) {
-    const int sl = r * G::NG + rg;
-    const int i = KC ? sl : S.row_perm()[sl];
-    const float kr = S.k()[i], qr = S.q()[i], M = msh[sl];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      T[r][p] = __ffma2_rn(T[r][p], f2(M), __fmul2_rn(f2(kr), W[p]));
-      part[p] = r == 0 ? __fmul2_rn(T[r][p], f2(qr)) : __ffma2_rn(T[r][p], f2(qr), part[p]);
-    }
-  }
-  st |= requant_group<D, KC, G::RPT>(rec, S.row_off(), S.row_code(), S.row_perm(), S.phi(), 0, rg, cc, T);
-  column_deposit<D>(reinterpret_cast<float*>(red), rg, cc, part);
-  if (!DIRECT) fence_proxy_async_smem();  // the new record is read by the bulk store
-  __syncthreads();  // B3: the o partials and the new record are complete
-
-  {
-    const float O = column_total<D>(reinterpret_cast<const float*>(red));
-    if ((tid & 1) == 0) {
-      const int j = tid >> 1;
-      const float oj = __fmul_rn(S.c()[j], O);
-      if (oj != oj) st |= ST_NAN;
-      o[j] = oj;
-    }
-  }
-  mbar_arrive(free_bar);  // this thread is done with the o partials
-  if (tid == 0) {
-    if (!DIRECT) {
-      bulk_s2g(hd->dst, S.rec(), hd->bytes);
-      bulk_commit();
-    }
-    pr->pend = sidx;
-  }
-  return true;
-}
-
-template <int D>
-__global__ void __launch_bounds__(Geo<D>::NT, 2) k_decode_step_packed(const StepArgs a) {
-  using G = Geo<D>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bars[4];
-  __shared__ __align__(8) uint64_t free_bar;
-  __shared__ __align__(16) float wsh[D];
-  __shared__ __align__(16) float msh[D];
-  __shared__ Producer prod;
-  __shared__ uint32_t st_sh;
-  __shared__ int abort_sh;
-  // [S^T k / o partials: NG D fp64][stage 0][stage 1]...
-  uint8_t* red = smem;
-  uint8_t* stages = smem + (size_t)G::NG * D * 8;
-
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int cc = lane % G::LPR;
-  const int rg = warp * G::RPW + lane / G::LPR;
-
-  int ahead = 0;  // thread 0: the chunk claimed for after the current one
-  if (tid == 0) {
-    for (int s = 0; s < a.nstage; ++s) mbar_init(&bars[s], 1);
-    mbar_init(&free_bar, G::NT);
-    fence_mbar_init();
-    st_sh = 0;
-    abort_sh = 0;
-    producer_start(a, &prod, ahead);
-    for (int s = 0; s < a.nstage; ++s) issue_next<D>(a, &prod, stages, bars, s, ahead);
-  }
-  __syncthreads();
-
-  uint32_t st = 0;
-  int n = 0;
-  for (;; ++n) {
-    const int sidx = n % a.nstage;
-    const uint32_t parity = (uint32_t)(n / a.nstage) & 1u;
-    const Stage<D> S{stages + (size_t)sidx * a.stage_bytes, a.rec_cap};
-    // The header was written by thread 0 before at least one block barrier
-    // that every thread has passed since, so it is read without waiting for
-    // the stage's data; the control flow below is uniform over the CTA.
-    const int tile = S.hdr()->tile;  // b * h_v + h
-    if (tile < 0) break;
-    float* o = a.o + (size_t)tile * D;
-    if (!S.hdr()->valid) {
-      if (tid < D) o[tid] = 0.0f;
-      st |= ST_SLOT;
-      __syncthreads();  // every thread has read the header and finished the previous tile
-      mbar_arrive(&free_bar);
-      if (tid == 0) {
-        refill_pending<D>(a, &prod, stages, bars, ahead);
-        prod.pend = sidx;  // nothing was loaded or stored: refill at the next refill point
-      }
-      __syncthreads();  // publish the refilled header before its tile is read
-      continue;
-    }
-    bool ok;
-    switch (S.hdr()->kind) {
-      case 8:
-        ok = packed_tile<D, 8>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
-                               &prod, ahead, o, rg, cc, st);
-        break;
-      case 6:
-        ok = packed_tile<D, 6>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
-                               &prod, ahead, o, rg, cc, st);
-        break;
-      case 4:
-        ok = packed_tile<D, 4>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
-                               &prod, ahead, o, rg, cc, st);
-        break;
-      case 2:
-        ok = packed_tile<D, 2>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
-                               &prod, ahead, o, rg, cc, st);
-        break;
-      case ROW_PIVOT:
-        ok = packed_tile<D, ROW_PIVOT>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh,
-                                       &abort_sh, &prod, ahead, o, rg, cc, st);
-        break;
-      default:
-        ok = packed_tile<D, 0>(a, S, sidx, parity, n, bars, &free_bar, stages, red, wsh, msh, &abort_sh,
-                               &prod, ahead, o, rg, cc, st);
-        break;
-    }
-    if (!ok) {
-      st |= ST_TIMEOUT;
-      break;
-    }
-  }
-  if (st) atomicOr(&st_sh, st);
-  __syncthreads();
-  if (tid == 0) {
-    if (abort_sh) {
-      // give the loads still in flight (tiles n .. n + nstage - 2) a bounded
-      // chance to land before the CTA exits
-      for (int k = 0; k + 1 < a.nstage; ++k) {
-        const TileHdr* hd = Stage<D>{stages + (size_t)((n + k) % a.nstage) * a.stage_bytes, a.rec_cap}.hdr();
-        if (hd->tile >= 0 && hd->valid)
-          (void)mbar_wait_bounded(&bars[(n + k) % a.nstage], (uint32_t)((n + k) / a.nstage) & 1u, 1000000ull);
-      }
-    }
-    bulk_wait_all();
-    if (st_sh) atomicOr(a.t.status, st_sh);
-    // The last CTA to finish resets the chunk counter for the next launch
-    // (every CTA's claims are ordered before its count by the fence).
-    __threadfence();
-    if (atomicAdd(a.t.sched + 1, 1u) == gridDim.x - 1) {
-      atomicExch(a.t.sched, 0u);
-      atomicExch(a.t.sched + 1, 0u);
-    }
-  }
 }
 
 // ===================================================== quantize / dequantize

@@ -165,3 +165,17 @@ class StatePool:
 
     def get_status(self, clear=True, stream=None) -> int:
         return _abi.sq_get_status(self._h, _stream(stream), clear)
+
+    def exact_count(self, clear=True, stream=None) -> int:
+        """Columns whose S^T k the packed steps summed exactly since the last clear."""
+        return _abi.sq_get_exact_count(self._h, _stream(stream), clear)
+
+    def launch_plan(self) -> dict:
+        return _abi.sq_launch_plan(self._h)
+
+    def set_wait_limit(self, ns: int) -> None:
+        _abi.sq_set_wait_limit(self._h, ns)
+
+    def test_stall_stages(self, extra_bytes: int) -> None:
+        """Testing only: make CTA 0's waits run out (see include/sq.h)."""
+        _abi.sq_test_stall_stages(self._h, extra_bytes)

@@ -151,7 +151,7 @@ def _coarse_rows(rng, p: Probe, rows, widths, pivot_rows=()):
 
 
 def near_probe(rng, d, widths=(8,), pivot_rows=(), fine_width=None,
-               rel=(2.0 ** -30, 2.0 ** -36, 2.0 ** -40, 2.0 ** -44), cancel=0, gate=None):
+               rel=(2.0 ** -30, 2.0 ** -36, 2.0 ** -40, 2.0 ** -44), cancel=0, gate=None, all_pivot=False):
     """Columns 0 .. d/2 - 2 sit about rel |P| on either side of an fp32
     midpoint (the fine row's own fp32 rounding moves that by at most
     2^-47 |P|; the exact sum is recomputed from the stored values, so the
@@ -163,12 +163,17 @@ def near_probe(rng, d, widths=(8,), pivot_rows=(), fine_width=None,
     fw = int(fine_width or widths[0])
     # gate: None -> a random value in [0.5, 1) per head (GDN) or per row, so
     # that r g has a full fp32 significand and V r g k needs up to 55 bits
+    if all_pivot:
+        pivot_rows = tuple(range(half))
     if gate is None:
-        p.g[:] = np.float32(rng.uniform(0.5, 1.0)) if len(widths) == 1 and not pivot_rows else \
+        p.g[:] = np.float32(rng.uniform(0.5, 1.0)) if (len(widths) == 1 and not pivot_rows) or all_pivot else \
             rng.uniform(0.5, 1.0, d).astype(np.float32)
     else:
         p.g[:] = np.float32(gate)
     _coarse_rows(rng, p, range(half), widths, pivot_rows)
+    if all_pivot:  # every row an fp16 pivot row (a GDN pivot head)
+        p.pivot[:] = True
+        p.scale[:] = 1.0
     # cancel > 0: rows c and half - 1 - c, c < cancel, get one large weight
     # and opposite codes, so their contributions cancel exactly in every
     # column; the other coarse rows are added between them in row order
@@ -190,7 +195,10 @@ def near_probe(rng, d, widths=(8,), pivot_rows=(), fine_width=None,
         j = t
         p.scale[f] = 1.0
         p.g[f] = p.g[0] if len(set(p.g.tolist())) == 1 else np.float32(1.0)
-        p.codes[f, j] = 1
+        if all_pivot:
+            p.half[f, j] = 1.0
+        else:
+            p.codes[f, j] = 1
         N, E = exact_sum((p.V(i, j), p.M(i), float(p.k[i])) for i in range(half))
         mN, mE = nearest_midpoint(N, E)
         e0 = min(mE, E)
@@ -250,9 +258,9 @@ def calib_for(probes, gate_kind):
     d = probes[0].d
     if gate_kind == 0:
         for p in probes:
-            assert not p.pivot.any() and len(set(p.width.tolist())) == 1
+            assert p.pivot.all() or (not p.pivot.any() and len(set(p.width.tolist())) == 1)
         bits = np.array([p.width[0] for p in probes], np.int8)
-        piv = np.zeros(h_v, np.uint8)
+        piv = np.array([p.pivot.all() for p in probes], np.uint8)
     else:
         bits = np.stack([p.width for p in probes]).astype(np.int8)
         piv = np.stack([p.pivot for p in probes]).astype(np.uint8)
