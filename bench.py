@@ -40,7 +40,12 @@ sys.path.insert(0, ROOT)
 METRIC = "quantized-state decode (request·head)-steps/s; achieved HBM GB/s vs B200 peak"
 UNIT = "(request*head)-steps/s"
 CONFIG_ID = 3
+# single-layer step workloads: the serving scale (the headline) and the
+# three smaller configurations, whose pools fit the 126 MB L2
+STEP_WORKLOADS = {"serving": 3, "plumbing": 0, "gdn_layer": 1, "kda_layer": 2}
 FALLBACK_HBM_GBS = 6650.0
+DATASHEET_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
 
 
 def peaks():
@@ -51,12 +56,29 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_config(w):
+def workload_config(w, pool_bytes=None):
     c = w.cfg
-    return {"workload": c.name, "batch_per_gpu": c.batch, "h_v": c.h_v, "h_k": c.h_k, "d": c.d,
-            "gate": "GDN (one gate per head)", "widths": "per-head {4,6,8}, 6-bit nominal, 5% FP16 pivot heads",
-            "warmup": f"{c.warmup_steps} unquantized steps, 2% outlier columns x20",
-            "l2": "state 222 MB > 126 MB L2 (no flush); 8 rotating input sets"}
+    if c.gate_kind == 0:
+        gate = "GDN (one gate per head)"
+        units = "per-head"
+    else:
+        gate = "KDA (one gate per key channel)"
+        units = "per-key-row"
+    widths = f"{units} {{{','.join(str(b) for b in c.widths)}}}, {c.nominal_bits}-bit nominal"
+    if c.pivot_frac:
+        widths += f", {round(100 * c.pivot_frac)}% FP16 pivot {'heads' if c.gate_kind == 0 else 'rows'}"
+    cfg = {"workload": c.name, "batch_per_gpu": w.B, "h_v": c.h_v, "h_k": c.h_k, "d": c.d, "gate": gate,
+           "widths": widths}
+    if c.warmup_steps:
+        cfg["warmup"] = f"{c.warmup_steps} unquantized steps, {round(100 * c.outlier_frac)}% outlier columns x20"
+    if pool_bytes is not None:
+        mb = pool_bytes / 1e6
+        if pool_bytes > L2_BYTES:
+            cfg["l2"] = f"state {mb:.0f} MB > 126 MB L2 (no flush); 8 rotating input sets"
+        else:
+            cfg["l2"] = (f"L2-resident: state {mb:.1f} MB < 126 MB L2, so the step runs from L2 "
+                         f"(no HBM roofline claim; GB/s below are algorithmic bytes over time)")
+    return cfg
 
 
 # ------------------------------------------------------------------ clocks
@@ -112,7 +134,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rank, world, local_rank, cid=CONFIG_ID):
     import torch
     from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
     from quantized_linear_attention_sq_b200.state import StatePool
@@ -124,7 +146,7 @@ def run_ours(args, rank, world, local_rank):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    w = synth.workload(CONFIG_ID, seed=shards.rank_seed(args.seed, rank))   # each rank: its own 512 requests
+    w = synth.workload(cid, seed=shards.rank_seed(args.seed, rank))   # each rank: its own requests
     c = w.cfg
     cal = w.calib()
     B = c.batch
@@ -141,7 +163,8 @@ def run_ours(args, rank, world, local_rank):
     for t in range(-c.warmup_steps, 0):
         q, k, v, beta, g = (torch.from_numpy(x).to(dev) for x in w.step_inputs(t))
         fp.decode_step(S, q, k, v, beta, g, o)
-    S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
+    if c.outlier_frac:
+        S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
     sp = make(_abi.SQ_FMT_PACKED)
     pool = sp.new_pool()
     clip = clip_fraction(S, cal, c)
@@ -238,17 +261,19 @@ def run_ours(args, rank, world, local_rank):
     achieved = bytes_launch / (kern_ms / 1e3) / 1e9
     fp_bytes = B * frep["state_bytes_per_step"]
     fp_kern = statistics.mean(fp_per)
+    l2_resident = B * rep["slot_bytes"] <= L2_BYTES
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
-        "config": workload_config(w),
+        "config": workload_config(w, B * rep["slot_bytes"]),
         "e2e": {"value": shards.job_rate(units, args.steps, e2e_ms, world), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "k_decode_step_packed<128>", "algorithmic_bytes_per_launch": bytes_launch,
+        "roofline": {"bound": "l2" if l2_resident else "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "frac_of_datasheet_8tbs": achieved / DATASHEET_HBM_GBS,
+                     "traffic": profiled_traffic() if cid == CONFIG_ID else None,
+                     "kernel": f"k_decode_step_packed<{c.d}>", "algorithmic_bytes_per_launch": bytes_launch,
                      "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
                   "clip_fraction": clip,
@@ -262,7 +287,9 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args, target_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(args, target_s=args.cpu_seconds, cid=cid)
+        one = cpu_baseline(args, target_s=max(2.0, args.cpu_seconds / 4), cid=cid, cores=1)
+        out["cpu_baseline"]["single_core"] = {"value": one["value"], "unit": UNIT, "sample": one["sample"]}
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -320,7 +347,7 @@ def clip_fraction(S, cal, c):
 
 
 # ------------------------------------------------------- the CPU oracle
-def cpu_baseline(args, target_s=15.0, steps=None):
+def cpu_baseline(args, target_s=15.0, steps=None, cid=CONFIG_ID, cores=None):
     """Time the CPU oracle (as it stands) on a bounded sample of the
     workload, tiles split over all host cores: a short probe measures the
     oracle's rate on this host, then `steps` decode steps (default: as many
@@ -329,17 +356,18 @@ def cpu_baseline(args, target_s=15.0, steps=None):
     import oracle
     from quantized_linear_attention_sq_b200 import synth
 
-    w = synth.workload(CONFIG_ID, seed=args.seed)
+    w = synth.workload(cid, seed=args.seed)
     c = w.cfg
     cal = w.calib()
-    cores = oracle.cores_available()
+    cores = cores or oracle.cores_available()
 
     def setup(reqs):
         o_ = oracle.Oracle(len(reqs), c.h_v, c.h_k, c.d, c.gate_kind, cal.unit_bits, cal.pivot, cal.col_scale,
                            cal.row_impact)
         pool = o_.new_pool()
         S = w.initial_state(reqs)
-        S *= w.outlier_mask()[None, :, None, :]
+        if c.outlier_frac:
+            S *= w.outlier_mask()[None, :, None, :]
         o_.quantize(pool, S)
         return o_, pool
 
@@ -373,25 +401,38 @@ def run_reference(args, rank, world):
     # each of the --steps steps is a bounded sample of the workload; the whole
     # run is sized to 4 x --cpu-seconds of CPU time (a minute by default)
     cb = cpu_baseline(args, target_s=4.0 * args.cpu_seconds, steps=max(1, args.steps))
+    import oracle
     from quantized_linear_attention_sq_b200 import synth
     w = synth.workload(CONFIG_ID, seed=args.seed)
+    cal = w.calib()
+    c = w.cfg
+    slot_bytes = oracle.Oracle(1, c.h_v, c.h_k, c.d, c.gate_kind, cal.unit_bits, cal.pivot, cal.col_scale,
+                               cal.row_impact).layout.slot_bytes
     full_step_ms = 1e3 * w.cfg.batch * w.cfg.h_v / cb["value"]  # one whole-batch step at the sample's rate
     out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_step_ms,
            "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, no dataset)",
-           "config": workload_config(w), "cpu_baseline": cb,
+           "config": workload_config(w, w.B * slot_bytes), "cpu_baseline": cb,
            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
            "note": "reference arm = the plain CPU oracle of the same step (no upstream code exists to install)"}
     print(json.dumps(out), flush=True)
 
 
-# ------------------------------------------- 8-layer KDA rollout (CUDA graph)
+# ------------------------------------------- 8-layer KDA rollout
 def run_rollout(args, rank, world, local_rank):
     """The long-rollout workload (8 KDA layers, 256 requests x 32 heads per
-    GPU, widths {2,4,6} at 4-bit nominal): one token = one step of every
-    layer. Timed with per-layer launches and with one CUDA graph holding 4
-    tokens x 8 layers of launches (prints its own JSON line)."""
+    GPU, per-row widths {2,4,6} at 4-bit nominal, 3 % FP16 pivot rows): one
+    token = one step of every layer. Two parts, one JSON line:
+      - the full rollout: 2048 tokens with inputs drawn on the device for
+        every layer and token; the quantized step of each token is timed
+        with CUDA events (input drawing excluded); the same inputs drive the
+        FP32-state step of every layer, and every 256 tokens the dequantized
+        quantized state is compared with the FP32 state (relative
+        Frobenius, per layer and over all layers: the drift of the
+        quantized rollout);
+      - launch overhead: per-layer launches vs one CUDA graph holding 4
+        tokens x 8 layers of launches, on 4 recycled input sets."""
     import torch
     from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
     from quantized_linear_attention_sq_b200.rollout import LayerStack
@@ -405,30 +446,75 @@ def run_rollout(args, rank, world, local_rank):
     works = [synth.workload(cid, seed=shards.rank_seed(args.seed, rank), layer=l) for l in range(nl)]
     c = works[0].cfg
     B = c.batch
-    layers, pools = [], []
+    layers, pools, fps, fstates = [], [], [], []
     for w in works:
         cal = w.calib()
         fp = StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, _abi.SQ_FMT_FP32)
         S = torch.from_numpy(w.initial_state()).to(dev)
         o = torch.empty((B, c.h_v, c.d), device=dev)
         for t in range(-c.warmup_steps, 0):
-            fp.decode_step(S, *(torch.from_numpy(x).to(dev) for x in w.step_inputs(t)), o)
+            fp.decode_step(S, *w.step_inputs_device(t), o)
         S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
         sp = StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, _abi.SQ_FMT_PACKED, cal.unit_bits, cal.pivot,
                        cal.col_scale, cal.row_impact)
         pool = sp.new_pool()
         sp.quantize_state(pool, S)
         torch.cuda.synchronize()
-        del S
-        fp.close()
         layers.append(sp)
         pools.append(pool)
+        fps.append(fp)
+        fstates.append(S)   # the FP32-state rollout starts from the same state
+    stream = torch.cuda.current_stream()
+    units = B * c.h_v * nl
+    bytes_token = sum(B * sp.report["state_bytes_per_step"] for sp in layers)
+    peak, peak_kind = peaks()
+
+    # ---- the full rollout with its drift
+    n_tok = c.steps
+    outs = [torch.empty((B, c.h_v, c.d), device=dev) for _ in works]
+    ofp = torch.empty((B, c.h_v, c.d), device=dev)
+    deq = torch.empty((B, c.h_v, c.d, c.d), device=dev)
+
+    def drift():
+        num = den = 0.0
+        per = []
+        for sp, pool, S in zip(layers, pools, fstates):
+            sp.dequantize_state(pool, deq)
+            dn = float(torch.linalg.vector_norm(deq - S)) ** 2
+            dd = float(torch.linalg.vector_norm(S)) ** 2
+            per.append((dn / dd) ** 0.5)
+            num += dn
+            den += dd
+        return (num / den) ** 0.5, per
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_tok)]
+    curve = []
+    with ClockSampler(local_rank) as clk:
+        for t in range(n_tok):
+            xs = [w.step_inputs_device(t) for w in works]
+            ev[t][0].record(stream)
+            for sp, pool, x, o in zip(layers, pools, xs, outs):
+                sp.decode_step(pool, *x, o)
+            ev[t][1].record(stream)
+            for fp, S, x in zip(fps, fstates, xs):
+                fp.decode_step(S, *x, ofp)
+            if (t + 1) % 256 == 0:
+                tot, per = drift()
+                curve.append({"step": t + 1, "rel_frobenius": tot, "per_layer": per})
+    clocks = clk.summary()
+    torch.cuda.synchronize()
+    roll_ms = sum(a.elapsed_time(b) for a, b in ev)
+    status = [sp.get_status() for sp in layers]
+    for fp in fps:
+        fp.close()
+    del fstates
+
+    # ---- launch overhead: eager per-layer launches vs one CUDA graph
     stack = LayerStack(layers)
     NI = 4
-    inputs = [[[torch.from_numpy(x).to(dev) for x in w.step_inputs(t)] for w in works] for t in range(NI)]
-    outs = [[torch.empty((B, c.h_v, c.d), device=dev) for _ in works] for _ in range(NI)]
+    inputs = [[list(w.step_inputs_device(10_000 + t)) for w in works] for t in range(NI)]
+    outs4 = [[torch.empty((B, c.h_v, c.d), device=dev) for _ in works] for _ in range(NI)]
     K = max(NI, args.steps // NI * NI)
-    stream = torch.cuda.current_stream()
 
     def timed(fn, reps):
         for _ in range(args.warmup):
@@ -444,28 +530,26 @@ def run_rollout(args, rank, world, local_rank):
 
     def eager_block():
         for t in range(NI):
-            stack.step(pools, inputs[t], outs[t])
+            stack.step(pools, inputs[t], outs4[t])
 
     eager_ms = timed(eager_block, K // NI)
-    graph = stack.capture(pools, inputs, outs)
+    graph = stack.capture(pools, inputs, outs4)
     graph_ms = timed(graph.replay, K // NI)
-    status = [sp.get_status() for sp in layers]
-    units = B * c.h_v * nl
-    bytes_token = sum(B * sp.report["state_bytes_per_step"] for sp in layers)
-    peak, peak_kind = peaks()
     out = {"metric": "8-layer KDA rollout (request*head*layer)-steps/s", "unit": "(request*head*layer)-steps/s",
-           "n_gpus": world, "tokens": K, "warmup_blocks": args.warmup,
+           "value": units * n_tok / (roll_ms / 1e3), "n_gpus": world, "higher_is_better": True,
            "config": {"workload": c.name, "batch_per_gpu": B, "h_v": c.h_v, "d": c.d, "layers": nl,
                       "gate": "KDA (one gate per key channel)",
-                      "widths": "per-row {2,4,6}, 4-bit nominal, 3% FP16 pivot rows"},
-           "eager": {"value": units * K / (eager_ms / 1e3), "ms_per_token": eager_ms / K,
-                     "launches_per_token": nl},
-           "graph": {"value": units * K / (graph_ms / 1e3), "ms_per_token": graph_ms / K,
-                     "tokens_per_replay": NI, "launches_per_replay": NI * nl},
-           "graph_speedup": eager_ms / graph_ms,
-           "achieved_gbs_graph": bytes_token / (graph_ms / K / 1e3) / 1e9,
-           "frac_graph": bytes_token / (graph_ms / K / 1e3) / 1e9 / peak,
-           "peak_kind": f"{peak_kind} hbm_gbs (copy)", "status_bits": status}
+                      "widths": "per-row {2,4,6}, 4-bit nominal, 3% FP16 pivot rows",
+                      "inputs": "drawn on the device per layer and token (Philox, seeded)"},
+           "rollout": {"tokens": n_tok, "ms_per_token": roll_ms / n_tok,
+                       "achieved_gbs": bytes_token / (roll_ms / n_tok / 1e3) / 1e9,
+                       "frac": bytes_token / (roll_ms / n_tok / 1e3) / 1e9 / peak,
+                       "drift_vs_fp32_state": curve, "clocks": clocks, "status_bits": status},
+           "launch_overhead": {
+               "eager": {"ms_per_token": eager_ms / K, "launches_per_token": nl},
+               "graph": {"ms_per_token": graph_ms / K, "tokens_per_replay": NI, "launches_per_replay": NI * nl},
+               "graph_speedup": eager_ms / graph_ms},
+           "peak_kind": f"{peak_kind} hbm_gbs (copy)"}
     del graph
     stack.close()
     if rank == 0:
@@ -601,12 +685,13 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["serving", "kda_rollout_8layers", "calibration", "prefill"],
+    ap.add_argument("--workload", choices=list(STEP_WORKLOADS) + ["kda_rollout_8layers", "calibration", "prefill"],
                     default="serving",
-                    help="serving: the headline GDN workload; kda_rollout_8layers: 8 KDA layers, "
-                         "per-layer launches vs one CUDA graph; calibration: the trace pass of the "
-                         "calibration library on the serving layer's shape; prefill: the prefill "
-                         "handoff on the serving shape")
+                    help="serving: the headline GDN workload (batch 512); plumbing, gdn_layer, kda_layer: "
+                         "the smaller L2-resident configurations; kda_rollout_8layers: 8 KDA layers, "
+                         "2048 steps with the drift against the FP32-state path, plus per-layer launches "
+                         "vs one CUDA graph; calibration: the trace pass of the calibration library on "
+                         "the serving layer's shape; prefill: the prefill handoff on the serving shape")
     ap.add_argument("--trace-samples", type=int, default=512,
                     help="calibration workload: state samples in the trace (512 = 1 GiB)")
     ap.add_argument("--prompt-len", type=int, default=128, help="prefill workload: tokens per prompt")
@@ -631,7 +716,7 @@ def main():
     elif args.workload == "prefill":
         run_prefill(args, rank, world, local_rank)
     else:
-        run_ours(args, rank, world, local_rank)
+        run_ours(args, rank, world, local_rank, cid=STEP_WORKLOADS[args.workload])
 
 
 if __name__ == "__main__":

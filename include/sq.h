@@ -242,12 +242,13 @@ sq_status sq_get_exact_count(sq_handle* h, void* stream, uint32_t* count, int32_
  * SQ_STATUS_TIMEOUT. */
 sq_status sq_set_wait_limit(sq_handle* h, uint64_t ns);
 
-/* Testing only (no passage). From the next packed decode step on, CTA 0 of
- * each launch makes every stage it fills expect `extra_bytes` (at most
- * 65536) more bytes than it loads, so its first wait runs out after the wait
- * limit: the step sets SQ_STATUS_TIMEOUT, writes no part of the tiles CTA 0
- * had taken, and the other CTAs finish the rest. 0 restores normal
- * operation. Every copy CTA 0 issues still lands; nothing is left in flight. */
+/* Testing only (no passage). From the next packed decode step on, the
+ * shared-memory stage that receives tile (request 0, head 0) expects
+ * `extra_bytes` (at most 65536) more bytes than are loaded into it, so the
+ * wait of the CTA that took that tile runs out after the wait limit: the
+ * step sets SQ_STATUS_TIMEOUT, that CTA leaves without writing any part of
+ * the tiles it had taken, and the other CTAs finish the rest. 0 restores
+ * normal operation. Every copy issued still lands; nothing is left in flight. */
 sq_status sq_test_stall_stages(sq_handle* h, uint32_t extra_bytes);
 
 /* Plumbing (no passage). Launch configuration of this handle's decode step
@@ -278,8 +279,11 @@ uint64_t sq_launch_count(const sq_handle* h);
  *     must fit the array (h_v * d <= 8192 always does); larger shapes are
  *     rejected with SQ_ERR_UNSUPPORTED and a message;
  *   - the first call on a device looks up the array's device address and
- *     sets the kernels' shared-memory limit for that device; make that
- *     first call before any stream capture;
+ *     sets the kernels' shared-memory limit for that device;
+ *   - the tables reach the array by an asynchronous copy from a host
+ *     buffer that every call overwrites, so the call must not be made while
+ *     `stream` is being captured into a CUDA graph: it then returns
+ *     SQ_ERR_UNSUPPORTED and launches nothing;
  *   - every call shares the one array, which keeps the last call's tables:
  *     calls on the same device serialize on the host, but calls whose GPU
  *     work overlaps (different streams, or a later call before the earlier

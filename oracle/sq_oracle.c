@@ -162,52 +162,44 @@ uint16_t sqo_f16_ru(float x) {
 
 /* --------------------------------------------------------- exact sums */
 /* A sum of products of floats, held exactly. Every finite float is an
- * integer significand times a power of two (frexp gives x = f 2^e with
- * f in [0.5, 1); f 2^24 is an integer for any float, subnormals included),
- * so a product of up to three floats is an integer below 2^72 times a power
- * of two. The accumulator is a two's complement fixed-point number of
- * XA_LIMBS 32-bit limbs whose bit 0 has weight 2^XA_LSB; that covers every
- * product of three finite floats (smallest weight 2^(3 (-149 - 23)) =
- * 2^-516, largest below 2^(3 128)) with room for the carries of any
- * number of terms this file adds. Each limb is kept in an int64 and
- * normalised only at the end, so adding a term never loses a bit.
- * A term that is not finite (inf or NaN operand) switches the sum to the
- * IEEE result, which for such terms does not depend on the order. */
+ * integer significand (below 2^24) times a power of two (2^-149 at the
+ * least), so a product of up to three floats is an integer below 2^72 times
+ * 2^e with e >= -447. The accumulator is a two's complement fixed-point
+ * number of XA_LIMBS 32-bit limbs whose bit 0 has weight 2^XA_LSB; that
+ * covers every product of three finite floats (weights from 2^-447 to below
+ * 2^(3 128)) with room for the carries of any number of terms this file
+ * adds. Each limb is kept in an int64 and
+ * normalised only at the end, so adding a term never loses a bit. */
 #define XA_LIMBS 32
 #define XA_LSB (-544)
 
 typedef struct {
   int64_t limb[XA_LIMBS];
-  int nonfinite;
-  long double ieee; /* IEEE sum, used only when a term is not finite */
 } xacc;
 
 static void xacc_init(xacc *a) { memset(a, 0, sizeof *a); }
 
-/* significand and exponent of a finite float: x = m 2^e exactly, m >= 0 */
+/* significand and exponent of a finite float: |x| = m 2^e exactly, read
+ * from its IEEE-754 binary32 fields (subnormals: exponent field 0, no
+ * implicit bit) */
 static void split_f32(float x, uint64_t *m, int *e) {
-  int ex;
-  double f = frexp(fabs((double)x), &ex);
-  *m = (uint64_t)ldexp(f, 24);
-  *e = ex - 24;
+  uint32_t b;
+  memcpy(&b, &x, 4);
+  uint32_t ef = (b >> 23) & 0xffu, fr = b & 0x7fffffu;
+  if (ef) { *m = fr | 0x800000u; *e = (int)ef - 150; }
+  else { *m = fr; *e = -149; }
 }
 
-/* a += x * y * z (pass z = 1 for a product of two) */
+/* a += x * y * z for finite x, y, z */
 static void xacc_add3(xacc *a, float x, float y, float z) {
-  if (!isfinite(x) || !isfinite(y) || !isfinite(z)) {
-    a->nonfinite = 1;
-    a->ieee += (long double)x * (long double)y * (long double)z;
-    return;
-  }
-  a->ieee += (long double)x * (long double)y * (long double)z;
   if (x == 0.0f || y == 0.0f || z == 0.0f) return;
   uint64_t mx, my, mz;
   int ex, ey, ez;
   split_f32(x, &mx, &ex);
   split_f32(y, &my, &ey);
   split_f32(z, &mz, &ez);
-  unsigned __int128 v = (unsigned __int128)mx * my * mz; /* < 2^72 */
-  int pos = ex + ey + ez - XA_LSB;                       /* bit index of v's bit 0 */
+  unsigned __int128 v = (unsigned __int128)(mx * my) * mz; /* < 2^72 */
+  int pos = ex + ey + ez - XA_LSB;                           /* bit index of v's bit 0, >= 544 - 447 */
   int neg = signbit(x) ^ signbit(y) ^ signbit(z);
   int li = pos / 32, sh = pos % 32;
   v <<= sh; /* < 2^103 */
@@ -232,7 +224,6 @@ static int limb_bit(const int64_t *l, int n) { return (int)((l[n / 32] >> (n % 3
  * subnormal quantum 2^-149 at the bottom and inf above the largest float;
  * an exact zero gives +0. */
 static float xacc_round_f32(const xacc *a) {
-  if (a->nonfinite) return (float)a->ieee;
   int64_t l[XA_LIMBS];
   memcpy(l, a->limb, sizeof l);
   xacc_normalise(l);
@@ -242,8 +233,12 @@ static float xacc_round_f32(const xacc *a) {
     xacc_normalise(l);
   }
   int top = -1; /* index of the most significant set bit */
-  for (int n = 32 * XA_LIMBS - 1; n >= 0; n--)
-    if (limb_bit(l, n)) { top = n; break; }
+  for (int i = XA_LIMBS - 1; i >= 0 && top < 0; i--)
+    if (l[i]) {
+      int b = 31;
+      while (!((l[i] >> b) & 1)) b--;
+      top = 32 * i + b;
+    }
   if (top < 0) return 0.0f;
   int qexp = top + XA_LSB - 23; /* exponent of the unit in the last place */
   if (qexp < -149) qexp = -149;
@@ -251,20 +246,40 @@ static float xacc_round_f32(const xacc *a) {
   uint64_t n = 0;
   for (int b = top; b >= q0 && b >= 0; b--) n = (n << 1) | (uint64_t)limb_bit(l, b);
   int half = q0 - 1 >= 0 ? limb_bit(l, q0 - 1) : 0;
-  int sticky = 0;
-  for (int b = q0 - 2; b >= 0 && !sticky; b--) sticky = limb_bit(l, b);
+  int sticky = 0; /* any set bit below the half bit */
+  int below = q0 - 1; /* bits 0 .. below-1 */
+  if (below > 0) {
+    int full = below / 32; /* limbs wholly below */
+    for (int i = 0; i < full && !sticky; i++) sticky = l[i] != 0;
+    int rem = below % 32;
+    if (!sticky && rem) sticky = (l[full] & (((int64_t)1 << rem) - 1)) != 0;
+  }
   if (half && (sticky || (n & 1))) n++;
   float r = (float)ldexp((double)n, qexp); /* exact, or inf beyond the largest float */
   return neg ? -r : r;
 }
 
+/* sum_i x[i*xs] y[i] z[i] of n terms (z NULL: all ones), exact and rounded
+ * once to fp32. A term with an inf or NaN factor makes the result the IEEE
+ * sum of the terms instead (inf, -inf or NaN, whatever the order). */
+static float exact_dot(const float *x, size_t xs, const float *y, const float *z, int n) {
+  for (int i = 0; i < n; i++)
+    if (!isfinite(x[i * xs]) || !isfinite(y[i]) || (z && !isfinite(z[i]))) {
+      long double s = 0.0L;
+      for (int t = 0; t < n; t++)
+        s += (long double)x[t * xs] * (long double)y[t] * (long double)(z ? z[t] : 1.0f);
+      return (float)s;
+    }
+  xacc a;
+  xacc_init(&a);
+  for (int i = 0; i < n; i++) xacc_add3(&a, x[i * xs], y[i], z ? z[i] : 1.0f);
+  return xacc_round_f32(&a);
+}
+
 /* sum_i x[i] y[i] z[i] exactly (z may be NULL: all ones), rounded once; an
  * entry point of its own so that the pins can check the exact sum directly */
 float sqo_exact_dot3(const float *x, const float *y, const float *z, int n) {
-  xacc a;
-  xacc_init(&a);
-  for (int i = 0; i < n; i++) xacc_add3(&a, x[i], y[i], z ? z[i] : 1.0f);
-  return xacc_round_f32(&a);
+  return exact_dot(x, 1, y, z, n);
 }
 
 /* -------------------------------------------------------------- layout */
@@ -444,10 +459,7 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
 
   load_VM(D, h, rec, gate, T, M);                      /* step 1 */
   for (int j = 0; j < d; j++) {                        /* steps 2-3 */
-    xacc acc;
-    xacc_init(&acc);
-    for (int i = 0; i < d; i++) xacc_add3(&acc, T[i * d + j], M[i], k[i]);
-    float P = xacc_round_f32(&acc);
+    float P = exact_dot(T + j, (size_t)d, M, k, d);
     float p = c[j] * P;
     float u = beta * (v[j] - p);
     float ic = 1.0f / c[j];
@@ -459,10 +471,7 @@ static uint32_t step_tile(const sqo_desc *D, uint8_t *rec, int b, int h,
       T[i * d + j] = fmaf(T[i * d + j], M[i], kw);
     }
   for (int j = 0; j < d; j++) {                        /* step 5 */
-    xacc acc;
-    xacc_init(&acc);
-    for (int i = 0; i < d; i++) xacc_add3(&acc, T[i * d + j], q[i], 1.0f);
-    float O = xacc_round_f32(&acc);
+    float O = exact_dot(T + j, (size_t)d, q, NULL, d);
     o[j] = c[j] * O;
     if (isnan(o[j])) st |= ST_NAN;
   }
@@ -585,19 +594,13 @@ uint32_t sqo_step_fp32_tiles(const sqo_desc *D, float *Spool, const float *q_all
     for (int i = 0; i < d; i++)
       for (int j = 0; j < d; j++) S[i * d + j] = gate[i] * S[i * d + j];
     for (int j = 0; j < d; j++) {
-      xacc acc;
-      xacc_init(&acc);
-      for (int i = 0; i < d; i++) xacc_add3(&acc, S[i * d + j], k[i], 1.0f);
-      float P = xacc_round_f32(&acc);
+      float P = exact_dot(S + j, (size_t)d, k, NULL, d);
       u[j] = beta * (v[j] - P);
     }
     for (int i = 0; i < d; i++)
       for (int j = 0; j < d; j++) S[i * d + j] = fmaf(k[i], u[j], S[i * d + j]);
     for (int j = 0; j < d; j++) {
-      xacc acc;
-      xacc_init(&acc);
-      for (int i = 0; i < d; i++) xacc_add3(&acc, S[i * d + j], q[i], 1.0f);
-      o[j] = xacc_round_f32(&acc);
+      o[j] = exact_dot(S + j, (size_t)d, q, NULL, d);
       if (isnan(o[j])) st |= ST_NAN;
     }
   }

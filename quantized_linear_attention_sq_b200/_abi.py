@@ -244,6 +244,8 @@ def sq_calib_allocate(sigma2, weight, widths, nominal_bits, pivot_frac):
     import numpy as np
     s2 = np.ascontiguousarray(sigma2, dtype=np.float64)
     w = np.ascontiguousarray(weight, dtype=np.float64)
+    if s2.ndim != 1 or w.ndim != 1 or s2.shape[0] != w.shape[0]:
+        raise ValueError(f"sigma2 and weight must be 1-D of one length (got {s2.shape} and {w.shape})")
     n = s2.shape[0]
     bits = np.zeros(n, np.int8)
     piv = np.zeros(n, np.uint8)

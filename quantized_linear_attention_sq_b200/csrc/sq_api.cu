@@ -192,7 +192,9 @@ sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int o
   const size_t static_smem = fa.sharedSizeBytes;
   const int nt = packed ? packed_threads_of(d) : threads_of(d);
   p->rec_cap = (uint32_t)round_up(stage_rec < 16 ? 16 : stage_rec, 128);
-  p->stage_bytes = packed ? (uint32_t)round_up(p->rec_cap + packed_aux_of(d), 128)
+  // packed: the record, 2 d bytes of slack (a row read of the widest kind
+  // from a clamped offset stays inside the stage), the vectors
+  p->stage_bytes = packed ? (uint32_t)round_up(p->rec_cap + 2u * d + packed_aux_of(d), 128)
                           : (uint32_t)round_up(p->rec_cap + 32u * d + 32u, 128);
   const size_t red = packed ? (size_t)16 * d * 8 : (size_t)32 * d * 4;
   const size_t dyn_max = (size_t)optin_smem - static_smem;
@@ -922,6 +924,17 @@ extern "C" sq_status sq_decode_step_noalloc(const sq_state_desc* desc, const sq_
     return fail(SQ_ERR_UNSUPPORTED, "no-alloc step: tables need %zu bytes, above its %zu-byte scratch", total,
                 kNoAllocScratchBytes);
 
+  // The tables travel by cudaMemcpyAsync from a host buffer that the next
+  // call overwrites. Captured into a CUDA graph, that copy would replay
+  // whatever tables the last call left there, so calls during a stream
+  // capture are refused.
+  {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t ce = cudaStreamIsCapturing(as_stream(stream), &cap);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaStreamIsCapturing");
+    if (cap != cudaStreamCaptureStatusNone)
+      return fail(SQ_ERR_UNSUPPORTED, "the no-alloc step cannot run while its stream is being captured");
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -65,7 +65,7 @@ struct StepArgs {
   uint32_t stage_bytes; // rec_cap + aux bytes, multiple of 128
   uint64_t slot_bytes;
   uint64_t wait_ns;     // limit of every bounded wait inside the kernel
-  uint32_t test_extra_tx;  // testing only: extra bytes CTA 0 expects per stage (0: none)
+  uint32_t test_extra_tx;  // testing only: extra bytes the stage of tile (request 0, head 0) expects (0: none)
   Tables t;
 };
 

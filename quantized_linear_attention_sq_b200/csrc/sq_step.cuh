@@ -49,6 +49,7 @@ struct PGeo {
   static constexpr int QS = RPT < 4 ? RPT : 4;  // rows requantized together
   // stage vectors: [k f32 D][q f32 D][g f32 D][phi f32 D][row_off u16 D]
   //                [row_code u8 D][row_perm u8 D][TileHdr 32 B], then the record
+  //                (rec_cap bytes) and 2 D bytes of slack
   static constexpr uint32_t AUX = (uint32_t)((20 * D + 32 + 127) / 128 * 128);
   static_assert(NT == D && RPT == LPR && RPT % QS == 0, "geometry");
 };
@@ -301,7 +302,7 @@ __device__ __forceinline__ void issue_pstage(const StepArgs& a, const TileScalar
   hd->g = x.g;
   hd->kind = x.kind;
   uint32_t tx = 3u * vec + (kda ? vec : 0u) + 3u * D + (mixed ? (uint32_t)D : 0u);
-  if (blockIdx.x == 0) tx += a.test_extra_tx;  // testing only: CTA 0's stages never complete
+  if (b == 0 && h == 0) tx += a.test_extra_tx;  // testing only: this stage never completes
   if (!direct) tx += x.rec_bytes;
   mbar_arrive_expect_tx(bar, tx);
   if (direct)
@@ -412,6 +413,60 @@ __device__ __forceinline__ void row_hi(const uint8_t* row, int cc, uint32_t (&xh
 }
 
 // -------------------------------------------------------------- pass B
+// 16 codes of width B (2, 4 or 6) as floats, reading most fields where they
+// lie: a field at bit s (s + B <= 23) of a source word X becomes the float
+// 2^23 + f 2^s by one AND-OR (X & (mask << s) | bits of 2^23), and one
+// f32x2 fma per pair, x 2^-s - (2^(23-s) + 2^(B-1)), gives the code exactly
+// (every intermediate is an integer below 2^24). The source words are the
+// chunk's words and a few shifts of them, chosen so that only two
+// (s, s') patterns occur among the pairs.
+template <int B>
+__device__ __forceinline__ uint32_t magic_at(uint32_t x, int s) {
+  return 0x4B000000u | (x & (((1u << B) - 1u) << s));
+}
+template <int B>
+__device__ __forceinline__ float2 code_pair(uint32_t x0, int s0, uint32_t x1, int s1) {
+  const float2 m = make_float2(__uint_as_float(magic_at<B>(x0, s0)), __uint_as_float(magic_at<B>(x1, s1)));
+  const float2 k = make_float2(1.0f / (float)(1u << s0), 1.0f / (float)(1u << s1));
+  const float2 c = make_float2(-(float)((1u << (23 - s0)) + (1u << (B - 1))),
+                               -(float)((1u << (23 - s1)) + (1u << (B - 1))));
+  return __ffma2_rn(m, k, c);
+}
+template <int B>
+__device__ __forceinline__ void unpack16_inplace(const uint32_t (&w)[B / 2], float2 (&V)[8]) {
+  if constexpr (B == 6) {
+    // 24-bit groups g (fields 4g .. 4g+3 at 0, 6, 12, 18); the field at 18
+    // comes from a second shift, at 6
+    const uint32_t G[4] = {w[0], __funnelshift_r(w[0], w[1], 24), __funnelshift_r(w[1], w[2], 16), w[2] >> 8};
+    const uint32_t H[4] = {w[0] >> 12, w[1] >> 4, __funnelshift_r(w[1], w[2], 28), w[2] >> 20};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      V[2 * g] = code_pair<6>(G[g], 0, G[g], 6);
+      V[2 * g + 1] = code_pair<6>(G[g], 12, H[g], 6);
+    }
+  } else if constexpr (B == 4) {
+    // per word: fields 0..3 at 0, 4, 8, 12 and fields 4..7 at the same
+    // places of the word shifted by 16
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t Y = w[k] >> 16;
+      V[4 * k] = code_pair<4>(w[k], 0, w[k], 4);
+      V[4 * k + 1] = code_pair<4>(w[k], 8, w[k], 12);
+      V[4 * k + 2] = code_pair<4>(Y, 0, Y, 4);
+      V[4 * k + 3] = code_pair<4>(Y, 8, Y, 12);
+    }
+  } else {
+    static_assert(B == 2, "widths 2, 4, 6");
+    // X_k = w >> 4k holds fields 2k, 2k+1 at 0, 2 and 2k+8, 2k+9 at 16, 18
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t X = w[0] >> (4 * k);
+      V[k] = code_pair<2>(X, 0, X, 2);
+      V[4 + k] = code_pair<2>(X, 16, X, 18);
+    }
+  }
+}
+
 // One row's 16 stored values as floats (codes, or fp16 values).
 template <int B, bool GLOBAL, bool VEC>
 __device__ __forceinline__ void row_values(const uint8_t* row, int cc, float2 (&V)[8]) {
@@ -435,7 +490,7 @@ __device__ __forceinline__ void row_values(const uint8_t* row, int cc, float2 (&
   } else {
     uint32_t w[B / 2];
     chunk_words<B, GLOBAL, VEC>(row, cc, w);
-    unpack16<B>(w, V);
+    unpack16_inplace<B>(w, V);
   }
 }
 
@@ -458,7 +513,7 @@ __device__ __forceinline__ float prow_absmax(const float2 (&t)[8]) {
 // Requantize the QS rows of group grp (row slots (grp QS + u) NG + rg):
 // one lane per row of the group computes the row scale, the others take it
 // by shuffle; new codes (or fp16 pivots) written into the record. A row
-// holding a NaN gets scale 0 and all codes 0.
+// holding a NaN gets scale 0 and all codes 0 (status bit NaN).
 template <int D, int KC, bool DIRECT>
 __device__ __forceinline__ uint32_t prequant(uint8_t* rec, const uint16_t* row_off, const uint8_t* row_code,
                                              const uint8_t* row_perm, const float* phi, uint32_t rec_cap, int grp,
@@ -492,9 +547,13 @@ __device__ __forceinline__ uint32_t prequant(uint8_t* rec, const uint16_t* row_o
     for (int u = 1; u < QS; ++u) mm = mine == u ? m[u] : mm;
     const int im = row_of(mine);
     const int cm = KC ? KC : row_code[im];
+    // A row holding a NaN keeps ir = lim = 0: every T' then clamps to +-0 (a
+    // NaN too: min.xorsign.abs returns its other operand) and rounds to code
+    // 0, with row scale 0.
     float ir_m = 0.0f, lim_m = 0.0f;
     if (cm != ROW_PIVOT) {
       uint16_t rbits = 0;
+      if (mm != mm) st |= ST_NAN;
       if (mm == mm) {
         const float qm = (float)((1 << (cm - 1)) - 1);
         const float s = __fdiv_rn(__fmul_rn(phi[im], mm), qm);
@@ -522,9 +581,6 @@ __device__ __forceinline__ uint32_t prequant(uint8_t* rec, const uint16_t* row_o
       uint8_t* row = row_ptr(i);
       if (code == ROW_PIVOT) {
         st |= store_row_pivot<false>(row, cc, T[u]);
-      } else if (m[u] != m[u]) {  // a NaN in the row (rare)
-        st |= ST_NAN;
-        store_row_zero(row, code, cc);
       } else if constexpr (KC != 0) {
         store_row_q<KC>(row, cc, ir, lim, T[u]);
       } else {
@@ -580,7 +636,11 @@ __device__ __forceinline__ float ptotal_f32(const float* red, int j) {
 // ------------------------------------------------------------ one tile
 // KC: width shared by every row of the head (ROW_PIVOT: all-pivot head, read
 // and written in place in the pool), or 0 for a head whose rows differ.
-// Returns false when a bounded wait gave up (the tile is abandoned). The
+// Returns false when a bounded wait gave up (the tile is abandoned: pass A
+// still runs, on stale shared memory, before the decision at B1; row
+// offsets of mixed-width heads are clamped to rec_cap, and a stage keeps
+// 2 D bytes after the record, so a row read of any width stays inside the
+// stage whatever the tables hold). The
 // loops over a thread's rows are not unrolled (per-row scalars come by
 // shuffle or from shared memory), which keeps each width's code small
 // enough for the instruction cache.

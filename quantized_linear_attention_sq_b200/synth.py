@@ -37,6 +37,7 @@ _STREAM_STATE = 1
 _STREAM_STEP = 2
 _STREAM_TRACE = 3
 _STREAM_PROMPT = 4
+_STREAM_DEVICE = 5
 
 
 @dataclass(frozen=True)
@@ -210,6 +211,32 @@ class Workload:
         C-contiguous.
         """
         return self._token_inputs(_STREAM_STEP, step, requests)
+
+    def step_inputs_device(self, step: int, device="cuda"):
+        """Inputs of decode step ``step`` for requests 0 .. B-1 drawn on the
+        device (for rollouts of thousands of steps, where drawing on the host
+        would take longer than the steps): the distributions of
+        ``step_inputs`` (q, k L2-normalised per head, v ~ N(0, 1), beta =
+        sigmoid(N(0, 1)), the workload's constant gates), from torch's
+        counter-based (Philox) generator seeded by (seed, config, layer,
+        step). Different values from ``step_inputs``; the same call always
+        gives the same values. Returns CUDA fp32 tensors q, k [B, h_k, d],
+        v [B, h_v, d], beta [B, h_v], g [B, h_v] or [B, h_v, d]."""
+        import torch
+        c = self.cfg
+        key = np.random.SeedSequence([self.seed, c.cid, self.layer, _STREAM_DEVICE, step + (1 << 20)])
+        gen = torch.Generator(device=device)
+        gen.manual_seed(int(key.generate_state(1, np.uint64)[0] >> 1))
+        B = self.B
+        q = torch.randn((B, c.h_k, c.d), generator=gen, device=device)
+        k = torch.randn((B, c.h_k, c.d), generator=gen, device=device)
+        q = (q / q.norm(dim=-1, keepdim=True)).contiguous()
+        k = (k / k.norm(dim=-1, keepdim=True)).contiguous()
+        v = torch.randn((B, c.h_v, c.d), generator=gen, device=device)
+        beta = torch.sigmoid(torch.randn((B, c.h_v), generator=gen, device=device))
+        gate = torch.from_numpy(self.calib().gate).to(device)
+        g = gate.expand((B,) + tuple(gate.shape)).contiguous()
+        return q, k, v, beta, g
 
     def _token_inputs(self, stream: int, step: int, requests):
         c = self.cfg

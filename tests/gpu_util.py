@@ -236,3 +236,64 @@ def free_rollout(w, o_, sp, init_ref, reqs, steps, inputs):
     r = rel_l2(S_gpu.cpu().numpy(), S_ref)
     sp2.close()
     return r
+
+
+def run_parity_device_inputs(w: synth.Workload, steps: int, check_requests, rollout_check=True):
+    """run_parity for long rollouts: the GPU steps all B requests with inputs
+    drawn on the device (``Workload.step_inputs_device``); the oracle steps
+    the requests in `check_requests` on host copies of their rows. Same
+    per-step comparison and teacher forcing as run_parity. After the last
+    step, returns also the relative Frobenius of the checked requests'
+    dequantized states (GPU vs oracle) and, when a flip was seen, of a free
+    rollout from the same start."""
+    c = w.cfg
+    B = w.B
+    reqs = list(check_requests)
+    sel = np.asarray(reqs)
+    sel_t = torch.as_tensor(reqs, device="cuda", dtype=torch.long)
+    o_ = oracle_for(oracle, w, n_slots=len(reqs))
+    sp = gpu_pool_for(w, B)
+    S_ref = oracle_warm_state(w, reqs)
+    S_gpu = gpu_warm_state(w)
+    S_gpu.index_copy_(0, sel_t, torch.from_numpy(S_ref).cuda())
+    pool_ref = o_.new_pool()
+    o_.quantize(pool_ref, S_ref)
+    pool = sp.new_pool()
+    sp.quantize_state(pool, S_gpu)
+    torch.cuda.synchronize()
+    del S_gpu
+    gslots = np.asarray(reqs, np.int32)
+    assert np.array_equal(slot_bytes(pool, sp, gslots), pool_ref)
+    init_ref = pool_ref.copy()
+    o_dev = torch.empty((B, c.h_v, c.d), device="cuda")
+    stats = Stats()
+    flips_seen = False
+    host_inputs = []
+    for t in range(steps):
+        x = w.step_inputs_device(t)
+        sp.decode_step(pool, *x, o_dev)
+        xs = [a.index_select(0, sel_t).cpu().numpy() for a in x]
+        if rollout_check:
+            host_inputs.append(xs)
+        o_ref, _ = o_.step(pool_ref, *xs, threads=THREADS)
+        got = slot_bytes(pool, sp, gslots)
+        f0 = stats.flips + stats.r_flips
+        compare_slots(o_, pool_ref, got, stats)
+        if stats.flips + stats.r_flips != f0:
+            flips_seen = True
+            p = pool.view(-1, sp.slot_bytes)
+            p[torch.as_tensor(gslots, device="cuda", dtype=torch.long)] = \
+                torch.from_numpy(pool_ref.reshape(len(reqs), -1)).cuda()
+        stats.worst_o = max(stats.worst_o, rel_l2(o_dev.index_select(0, sel_t).cpu().numpy(), o_ref))
+        stats.steps += 1
+    # final state of the checked requests: GPU vs oracle (equal unless flips)
+    S_g = torch.empty((len(reqs), c.h_v, c.d, c.d), device="cuda")
+    sp.dequantize_state(pool, S_g, torch.from_numpy(gslots).cuda())
+    S_o, _ = o_.dequantize(pool_ref)
+    final = rel_l2(S_g.cpu().numpy(), S_o)
+    rollout = 0.0
+    if flips_seen and rollout_check:
+        n = len(reqs)
+        rollout = free_rollout(w, o_, sp, init_ref, list(range(n)), steps, lambda t: host_inputs[t])
+    sp.close()
+    return stats, final, rollout

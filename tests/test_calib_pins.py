@@ -205,6 +205,14 @@ def _lib_alloc(sigma2, w, widths, nominal, pf):
     (2, 513, (2, 4, 6, 8), 5, 0.0),     # odd count, all four widths
     (3, 300, (4, 8), 6, 0.1),           # unequal raise sizes (4 -> 8)
     (4, 64, (2, 8), 2, 1.0),            # every unit a pivot
+    # raise sizes that differ (2 -> 4 costs 2 bits, 4 -> 8 costs 4; 2 -> 6
+    # costs 4, 6 -> 8 costs 2), at budgets that leave less than the larger
+    # raise: the rule that skips a raise too big for what is left decides
+    (5, 40, (2, 4, 8), 3, 0.0),
+    (6, 40, (2, 4, 8), 5, 0.05),
+    (7, 64, (2, 6, 8), 3, 0.0),
+    (8, 64, (2, 6, 8), 7, 0.1),
+    (9, 33, (2, 4, 8), 7, 0.0),
 ])
 def test_library_allocation_equals_oracle(seed, n, widths, nominal, pf):
     rng = np.random.default_rng(seed)
@@ -226,6 +234,13 @@ def test_library_allocation_ties_go_to_the_lower_index():
         got = _lib_alloc(sigma2, w, widths, nominal, pf)
         np.testing.assert_array_equal(got[1], want[1])
         np.testing.assert_array_equal(got[0], want[0])
+
+
+def test_library_allocation_rejects_mismatched_arrays():
+    with pytest.raises(ValueError, match="one length"):
+        _lib_alloc(np.ones(8), np.ones(7), (4, 6), 5, 0.0)
+    with pytest.raises(ValueError, match="one length"):
+        _lib_alloc(np.ones((2, 4)), np.ones(8), (4, 6), 5, 0.0)
 
 
 def test_library_allocation_rejects_bad_budgets_and_values():

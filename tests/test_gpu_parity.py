@@ -82,15 +82,19 @@ def test_layer_configs_full_batch_sampled(cid, reqs):
     assert rollout <= gu.ROLLOUT_TOL
 
 
-@pytest.mark.parametrize("layer", [0, 7])
-def test_long_rollout_config_sampled(layer):
-    """One KDA layer of the 8-layer, batch-256 workload at full batch; two
-    sampled requests followed for 512 steps."""
+@pytest.mark.parametrize("layer", range(8))
+def test_long_rollout_config_full(layer):
+    """The 8-layer, batch-256 KDA workload at its full length: every layer
+    steps all 256 requests for 2048 steps (inputs drawn on the device); the
+    oracle follows two requests per layer (a different pair per layer) with
+    the per-step acceptance, and their final dequantized states agree within
+    1e-3 relative Frobenius."""
     w = synth.workload(4, layer=layer)
-    stats, rollout = gu.run_parity(w, 512, check_requests=[3, 250], use_gpu_warmup=True)
-    _report(f"long_rollout_l{layer}", stats, rollout)
+    reqs = [(3 + 37 * layer) % 256, (250 - 29 * layer) % 256]
+    stats, final, rollout = gu.run_parity_device_inputs(w, w.cfg.steps, reqs)
+    _report(f"long_rollout_l{layer} reqs={reqs}", stats, max(final, rollout))
     stats.check()
-    assert rollout <= gu.ROLLOUT_TOL
+    assert final <= gu.ROLLOUT_TOL and rollout <= gu.ROLLOUT_TOL
 
 
 @pytest.mark.parametrize("d", [32, 64, 128])
