@@ -69,6 +69,10 @@ def lib():
             L.sqo_quantize.restype = ctypes.c_uint32
             L.sqo_dequantize.argtypes = [P, P, P, P, ctypes.c_int]
             L.sqo_dequantize.restype = ctypes.c_uint32
+            L.sqo_window_record_bytes.argtypes = [P, ctypes.c_int]
+            L.sqo_window_record_bytes.restype = ctypes.c_size_t
+            L.sqo_window_step_tiles.argtypes = [P, P, P, ctypes.c_int] + [P] * 7 + [ctypes.c_int, ctypes.c_int]
+            L.sqo_window_step_tiles.restype = ctypes.c_uint32
             _lib = L
         return _lib
 
@@ -164,6 +168,22 @@ class Oracle:
         ``tiles`` = (t0, t1) restricts the step to tiles t0 .. t1-1
         (tile = request * h_v + head); ``threads`` splits them over host threads."""
         return self._run_tiles(lib().sqo_step_tiles, pool, q, k, v, beta, g, slots, o, threads, tiles)
+
+    # ------------------------------------------- per-window variant
+    def window_record_bytes(self, W: int) -> int:
+        return lib().sqo_window_record_bytes(self._dp, W)
+
+    def new_window_buffer(self, W: int):
+        return np.zeros(self.n_slots * self.h_v * self.window_record_bytes(W), dtype=np.uint8)
+
+    def window_step(self, pool, wbuf, W, q, k, v, beta, g, slots=None, o=None, threads=1):
+        """One token of the per-window variant in place on pool and wbuf
+        (window records [n_slots][h_v]); returns (o, status)."""
+        fn = lib().sqo_window_step_tiles
+
+        def run(dp, state, *rest):
+            return fn(dp, state, _ptr(wbuf), W, *rest)
+        return self._run_tiles(run, pool, q, k, v, beta, g, slots, o, threads, None)
 
     def step_fp32(self, S, q, k, v, beta, g, slots=None, o=None, threads=1, tiles=None):
         """Unquantized step in place on the fp32 pool S [n_slots, h_v, d, d]."""

@@ -612,3 +612,136 @@ uint32_t sqo_step_fp32(const sqo_desc *D, float *Spool, const float *q, const fl
                        const float *beta, const float *g, float *o, const int32_t *slots, int B) {
   return sqo_step_fp32_tiles(D, Spool, q, k, v, beta, g, o, slots, 0, B * D->h_v);
 }
+
+/* ------------------------------------------------ per-window variant */
+/* Per-window quantization ("线性注意力每生成一个token都要搬状态，LeapQuant
+ * 把它压到8位还不掉点" (wink.run), the first of the three techniques): the
+ * packed state is not requantized after every token; it stays frozen for a
+ * window of W tokens, the tokens' updates are kept at high precision in a
+ * buffer, the outputs come from the frozen state and the buffer together,
+ * and at the end of the window the state is requantized once.
+ *
+ * Window buffer (this project's layout): per (slot, value head) a record of
+ * sqo_window_record_bytes() bytes: [int32 count, 12 pad bytes]
+ * [k: W x d fp32][u: W x d fp32][gates: W x gd fp32, padded to 16 B], gd = d
+ * for one gate per key channel, 1 for one per head. count tokens are
+ * buffered (0 <= count < W); token tau's key k_tau, its u_tau and its gate
+ * G_tau are stored at row tau.
+ *
+ * One token for a tile with n buffered tokens (current token = n), in fp64
+ * (every product and sum below in double; only u and o are rounded to
+ * fp32, u because the buffer stores it in fp32):
+ *   S0_ij = V_ij M_i c_j, the frozen state (V, M as in load_VM without gate)
+ *   D_tau,i = prod_{sigma = tau+1 .. n} G_sigma,i (tau = -1 .. n-1; D_-1
+ *            decays S0 through token n)
+ *   Sg_ij = D_-1,i S0_ij + sum_{tau<n} D_tau,i k_tau,i u_tau,j
+ *           (the state after the buffered tokens, gated by G_n)
+ *   p_j = sum_i Sg_ij k_n,i ; u_n,j = fp32(beta (v_j - p_j))
+ *   S_ij = Sg_ij + k_n,i u_n,j ; o_j = fp32(sum_i S_ij q_n,i)
+ * then token n is appended (count n + 1), and when count reaches W the
+ * state is requantized once, T'_ij = fp32(S_ij ic_j) with ic_j = fp32(1/c_j),
+ * by the step's requantization (store_T), and count returns to 0.
+ * A slot id out of range skips the tile (o = 0, status bit). */
+static size_t window_gate_floats(const sqo_desc *D, int W) {
+  size_t n = (size_t)W * (D->gate_kind == 0 ? 1 : (size_t)D->d);
+  return (n + 3) / 4 * 4;
+}
+size_t sqo_window_record_bytes(const sqo_desc *D, int W) {
+  return 16 + 4 * (2 * (size_t)W * D->d + window_gate_floats(D, W));
+}
+
+static uint32_t window_tile(const sqo_desc *D, uint8_t *rec, uint8_t *wrec, int W, int b, int h,
+                            const float *q_all, const float *k_all, const float *v_all,
+                            const float *beta_all, const float *g_all, float *o_all) {
+  int d = D->d;
+  int hk = h / (D->h_v / D->h_k);
+  const float *q = q_all + ((size_t)b * D->h_k + hk) * d;
+  const float *k = k_all + ((size_t)b * D->h_k + hk) * d;
+  const float *v = v_all + ((size_t)b * D->h_v + h) * d;
+  double beta = beta_all[(size_t)b * D->h_v + h];
+  float *o = o_all + ((size_t)b * D->h_v + h) * d;
+  const float *c = D->col_scale + (size_t)h * d;
+  int gd = D->gate_kind == 0 ? 1 : d;
+  int32_t n;
+  memcpy(&n, wrec, 4);
+  float *kb = (float *)(wrec + 16);
+  float *ub = kb + (size_t)W * d;
+  float *gb = ub + (size_t)W * d;
+  uint32_t st = 0;
+  float *V = malloc(sizeof(float) * d * d);
+  float *M = malloc(sizeof(float) * d);
+  double *S = malloc(sizeof(double) * d * d);
+  double *Dg = malloc(sizeof(double) * (W + 1) * d); /* Dg[(tau+1) d + i] = D_tau,i */
+  float *T = malloc(sizeof(float) * d * d);
+  load_VM(D, h, rec, NULL, V, M);
+  /* the current token's gate */
+  float *gcur = gb + (size_t)n * gd;
+  for (int x = 0; x < gd; x++) gcur[x] = D->gate_kind == 0 ? g_all[(size_t)b * D->h_v + h]
+                                                           : g_all[((size_t)b * D->h_v + h) * d + x];
+  for (int i = 0; i < d; i++) {
+    double acc = 1.0;
+    for (int tau = n - 1; tau >= -1; tau--) {
+      acc *= (double)gb[(size_t)(tau + 1) * gd + (gd == 1 ? 0 : i)];
+      Dg[(size_t)(tau + 1) * d + i] = acc;
+    }
+  }
+  for (int i = 0; i < d; i++)
+    for (int j = 0; j < d; j++) {
+      double s = Dg[i] * ((double)V[i * d + j] * (double)M[i] * (double)c[j]);
+      for (int tau = 0; tau < n; tau++)
+        s += Dg[(size_t)(tau + 1) * d + i] * (double)kb[(size_t)tau * d + i] * (double)ub[(size_t)tau * d + j];
+      S[i * d + j] = s;
+    }
+  float *un = ub + (size_t)n * d;
+  for (int j = 0; j < d; j++) {
+    double p = 0.0;
+    for (int i = 0; i < d; i++) p += S[i * d + j] * (double)k[i];
+    un[j] = (float)(beta * ((double)v[j] - p));
+  }
+  for (int i = 0; i < d; i++) kb[(size_t)n * d + i] = k[i];
+  for (int i = 0; i < d; i++)
+    for (int j = 0; j < d; j++) S[i * d + j] += (double)k[i] * (double)un[j];
+  for (int j = 0; j < d; j++) {
+    double acc = 0.0;
+    for (int i = 0; i < d; i++) acc += S[i * d + j] * (double)q[i];
+    o[j] = (float)acc;
+    if (isnan(o[j])) st |= ST_NAN;
+  }
+  n += 1;
+  if (n == W) {
+    for (int i = 0; i < d; i++)
+      for (int j = 0; j < d; j++) {
+        float ic = 1.0f / c[j];
+        T[i * d + j] = (float)(S[i * d + j] * (double)ic);
+      }
+    st |= store_T(D, h, rec, T);
+    n = 0;
+  }
+  memcpy(wrec, &n, 4);
+  free(V); free(M); free(S); free(Dg); free(T);
+  return st;
+}
+
+/* One token of the per-window variant for tiles [t0, t1) of a batch of B
+ * requests (inputs as in sqo_step_tiles); wbuf is [n_slots][h_v] window
+ * records. Returns the status bits. */
+uint32_t sqo_window_step_tiles(const sqo_desc *D, uint8_t *pool, uint8_t *wbuf, int W, const float *q,
+                               const float *k, const float *v, const float *beta, const float *g, float *o,
+                               const int32_t *slots, int t0, int t1) {
+  int d = D->d;
+  uint32_t st = 0;
+  size_t slot_bytes = sqo_slot_bytes(D);
+  size_t wrb = sqo_window_record_bytes(D, W);
+  for (int t = t0; t < t1; t++) {
+    int b = t / D->h_v, h = t % D->h_v;
+    int s = slot_of(D, slots, b, &st);
+    if (s < 0) {
+      memset(o + ((size_t)b * D->h_v + h) * d, 0, sizeof(float) * d);
+      continue;
+    }
+    uint8_t *rec = pool + (size_t)s * slot_bytes + sqo_head_offset(D, h);
+    uint8_t *wrec = wbuf + ((size_t)s * D->h_v + h) * wrb;
+    st |= window_tile(D, rec, wrec, W, b, h, q, k, v, beta, g, o);
+  }
+  return st;
+}
