@@ -259,6 +259,8 @@ __device__ __noinline__ float column_warp(const uint8_t* rec, const uint16_t* ro
   float P;
   if (!(fabs(s) <= 1.7976931348623157e308) || !(fabs(c) <= 1.7976931348623157e308)) {
     P = (float)(s + c);
+  } else if (mag == 0.0) {
+    P = 0.0f;  // every term is zero (e.g. a column whose codes are all 0): +0
   } else {
     const float flo = __double2float_rn(__dadd_rd(s, __dsub_rd(c, eps)));
     const float fhi = __double2float_rn(__dadd_ru(s, __dadd_ru(c, eps)));
