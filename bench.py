@@ -307,10 +307,12 @@ def profiled_traffic():
     rec_path = os.path.join(ROOT, "profiles", "k_decode_step_packed_gdn_serving_b512.traffic.json")
     try:
         rec = json.load(open(rec_path))
-        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
-    except (OSError, ValueError, KeyError):
+        h = hashlib.sha256()
+        for f in rec["sources"]:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+    except (OSError, ValueError, KeyError, TypeError):
         return None
-    if hashlib.sha256(src).hexdigest() != rec["kernel_source_sha256"]:
+    if h.hexdigest() != rec["kernel_source_sha256"]:
         return None
     return rec["dram_bytes_read"] + rec["dram_bytes_write"]
 
