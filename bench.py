@@ -320,31 +320,34 @@ def profiled_traffic():
 def clip_fraction(S, cal, c):
     """Share of the quantized rows' entries that the row scale clips when
     the state S [B, h_v, d, d] is quantized: |T_ij| / r_i rounds beyond qmax,
-    with T = S / c and r_i the fp16 round-up of phi_i max_j |T_ij| / qmax
-    (rows with phi_i < 1 clip their largest entries). GDN units (one width
-    per head); pivot heads are not counted."""
+    with T = S / c and r_i the fp16 round-up of min(phi_i, 1) max_j |T_ij| /
+    qmax_i (rows with phi_i < 1 clip their largest entries). Widths per head
+    (GDN) or per key row (KDA); pivot units are not counted."""
     import torch
 
     dev = S.device
-    keep = torch.from_numpy(cal.pivot == 0).to(dev)                           # [h_v]
-    qmax = torch.from_numpy((2.0 ** (cal.unit_bits.astype("float64") - 1) - 1).astype("float32")).to(dev)
-    ic = 1.0 / torch.from_numpy(cal.col_scale).to(dev)                         # [h_v, d]
-    phi = torch.from_numpy(cal.row_impact).to(dev)                             # [h_v, d]
+    h_v, d = c.h_v, c.d
+    bits = np.broadcast_to(cal.unit_bits.reshape(h_v, -1), (h_v, d)).astype("float64")
+    piv = np.broadcast_to(cal.pivot.reshape(h_v, -1), (h_v, d))
+    keep = torch.from_numpy(np.ascontiguousarray(piv == 0)).to(dev)                   # [h_v, d] rows
+    qmax = torch.from_numpy((2.0 ** (bits - 1) - 1).astype("float32")).to(dev)       # [h_v, d]
+    ic = 1.0 / torch.from_numpy(cal.col_scale).to(dev)                               # [h_v, d] columns
+    phi = torch.from_numpy(np.minimum(cal.row_impact, 1.0).astype("float32")).to(dev)  # [h_v, d] rows
     clipped = 0
     total = 0
-    for b0 in range(0, S.shape[0], 64):                                        # bounded temporaries
+    for b0 in range(0, S.shape[0], 64):                                              # bounded temporaries
         T = S[b0:b0 + 64] * ic[None, :, None, :]
-        m = T.abs().amax(dim=3)                                                # [b, h_v, d]
-        s = phi[None] * m / qmax[None, :, None]
+        m = T.abs().amax(dim=3)                                                      # [b, h_v, d]
+        s = phi[None] * m / qmax[None]
         h = s.to(torch.float16)
         up = (h.float() < s) & (h.float() < 65504)
-        h = torch.where(up, (h.view(torch.int16) + 1).view(torch.float16), h)   # round toward +inf
+        h = torch.where(up, (h.view(torch.int16) + 1).view(torch.float16), h)         # round toward +inf
         r = h.float()
-        lim = qmax[None, :, None, None] + 0.5
+        lim = qmax[None, :, :, None] + 0.5
         over = (T.abs() * (1.0 / r).unsqueeze(3)) > lim
-        over = over & keep[None, :, None, None] & (r > 0).unsqueeze(3)
+        over = over & keep[None, :, :, None] & (r > 0).unsqueeze(3)
         clipped += int(over.sum())
-        total += int(keep.sum()) * T.shape[0] * c.d * c.d
+        total += int(keep.sum()) * T.shape[0] * d
     return clipped / max(total, 1)
 
 
