@@ -299,6 +299,154 @@ def run_ours(args, rank, world, local_rank, cid=CONFIG_ID):
         print(json.dumps(out), flush=True)
 
 
+def run_window(args, rank, world, local_rank, cid=CONFIG_ID):
+    """The per-window variant (sq_window_step) on the serving workload:
+    W-token windows, timed over whole windows so that the share of
+    window-end requantizations is the variant's own (one token in W)."""
+    import torch
+    from quantized_linear_attention_sq_b200 import _abi, build, shards, synth
+    from quantized_linear_attention_sq_b200.state import StatePool
+
+    torch.cuda.set_device(local_rank)
+    build.build()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    W = args.window
+    w = synth.workload(cid, seed=shards.rank_seed(args.seed, rank))
+    c = w.cfg
+    cal = w.calib()
+    B = c.batch
+    dev = torch.device("cuda", local_rank)
+
+    def make(fmt):
+        return StatePool(B, c.h_v, c.h_k, c.d, c.gate_kind, fmt, cal.unit_bits, cal.pivot, cal.col_scale,
+                         cal.row_impact)
+
+    S = torch.from_numpy(w.initial_state()).to(dev)
+    fp = make(_abi.SQ_FMT_FP32)
+    o = torch.empty((B, c.h_v, c.d), device=dev)
+    for t in range(-c.warmup_steps, 0):
+        q, k, v, beta, g = (torch.from_numpy(x).to(dev) for x in w.step_inputs(t))
+        fp.decode_step(S, q, k, v, beta, g, o)
+    if c.outlier_frac:
+        S *= torch.from_numpy(w.outlier_mask()).to(dev)[None, :, None, :]
+    fp.close()
+    sp = make(_abi.SQ_FMT_PACKED)
+    pool = sp.new_pool()
+    sp.quantize_state(pool, S)
+    del S
+    wbuf = sp.new_window_buffer(W)
+    rec_w, buf_bytes = sp.window_buffer_bytes(W)
+    torch.cuda.synchronize()
+    setup_status = sp.get_status()
+    NI = 8
+    host_inputs = [w.step_inputs(t) for t in range(NI)]
+    dev_inputs = [[torch.from_numpy(x).to(dev) for x in xs] for xs in host_inputs]
+    stream = torch.cuda.current_stream()
+    if args.profile:
+        for i in range(args.profile):
+            sp.window_step(pool, wbuf, W, *dev_inputs[i % NI], o)
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_steps": args.profile, "window": W, "status_after_setup": setup_status,
+                          "status_bits": sp.get_status()}), flush=True)
+        sp.close()
+        return
+    K = max(W, args.steps // W * W)
+    Wm = max(W, (args.warmup + W - 1) // W * W)   # the timed region starts at a window's first token
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for i in range(Wm):
+        sp.window_step(pool, wbuf, W, *dev_inputs[i % NI], o)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    n0 = sp.launches()
+    props = torch.cuda.get_device_properties(local_rank)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank)
+    with ClockSampler(gpu_id) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            sp.window_step(pool, wbuf, W, *dev_inputs[i % NI], o)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    clocks = clk.summary()
+    launches = sp.launches() - n0
+    total_ms = shards.max_over_ranks(t0.elapsed_time(t1), dist, dev)
+    per = [a.elapsed_time(b) for a, b in ev]
+    kern_ms = statistics.mean(per)
+    end_ms = statistics.mean(per[W - 1::W])                       # window-end tokens
+    mid = [x for i, x in enumerate(per) if i % W != W - 1]
+    mid_ms = statistics.mean(mid) if mid else end_ms
+    # ---- end to end: pinned host inputs copied in, o copied out, every token
+    pinned = [[torch.from_numpy(x).pin_memory() for x in xs] for xs in host_inputs]
+    o_host = torch.empty((B, c.h_v, c.d), dtype=torch.float32).pin_memory()
+    stage = [torch.empty_like(x) for x in dev_inputs[0]]
+    h2d = sum(x.numel() * x.element_size() for x in pinned[0])
+    d2h = o_host.numel() * o_host.element_size()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for i in range(K):
+        for dst, src in zip(stage, pinned[i % NI]):
+            dst.copy_(src, non_blocking=True)
+        sp.window_step(pool, wbuf, W, *stage, o)
+        o_host.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = shards.max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    st_bits = sp.get_status()
+    rep = sp.report
+    gd = c.d if c.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1
+    # algorithmic bytes of one token, averaged over a window: the packed
+    # record read every token and written at the window's end, the buffered
+    # rows read (on average (W - 1) / 2 of them) and the token's row written
+    row = 4 * (2 * c.d + gd)
+    per_tile = rep["slot_bytes"] / c.h_v * (1 + 1 / W) + row * ((W - 1) / 2 + 1)
+    units = B * c.h_v
+    bytes_launch = units * per_tile
+    peak, peak_kind = peaks()
+    achieved = bytes_launch / (kern_ms / 1e3) / 1e9
+    cfg = workload_config(w, B * rep["slot_bytes"] + buf_bytes)
+    cfg["window"] = W
+    cfg["window_buffer_bytes"] = buf_bytes
+    out = {
+        "metric": METRIC, "value": shards.job_rate(units, K, total_ms, world), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic (seeded, no dataset)", "config": cfg,
+        "e2e": {"value": shards.job_rate(units, K, e2e_ms, world), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": f"k_window_step<{c.d}>",
+                     "algorithmic_bytes_per_launch": bytes_launch, "kernel_ms": kern_ms,
+                     "kernel_ms_inside_window": mid_ms, "kernel_ms_window_end": end_ms,
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+        "state": {"bits_per_value": rep["bits_per_value"], "status_after_setup": setup_status,
+                  "status_bits": st_bits},
+        "clocks": clocks,
+    }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    sp.close()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def profiled_traffic():
     """DRAM bytes (read + write) per launch of the packed step from the ncu
     capture recorded under profiles/, or None once the kernel source has
@@ -690,13 +838,17 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(STEP_WORKLOADS) + ["kda_rollout_8layers", "calibration", "prefill"],
+    ap.add_argument("--workload", choices=list(STEP_WORKLOADS) + ["kda_rollout_8layers", "calibration", "prefill",
+                                                                   "window_serving"],
                     default="serving",
                     help="serving: the headline GDN workload (batch 512); plumbing, gdn_layer, kda_layer: "
                          "the smaller L2-resident configurations; kda_rollout_8layers: 8 KDA layers, "
                          "2048 steps with the drift against the FP32-state path, plus per-layer launches "
                          "vs one CUDA graph; calibration: the trace pass of the calibration library on "
-                         "the serving layer's shape; prefill: the prefill handoff on the serving shape")
+                         "the serving layer's shape; prefill: the prefill handoff on the serving shape; "
+                         "window_serving: the per-window variant (--window tokens per window) on the "
+                         "serving workload")
+    ap.add_argument("--window", type=int, default=16, help="window_serving: tokens per window")
     ap.add_argument("--trace-samples", type=int, default=512,
                     help="calibration workload: state samples in the trace (512 = 1 GiB)")
     ap.add_argument("--prompt-len", type=int, default=128, help="prefill workload: tokens per prompt")
@@ -720,6 +872,8 @@ def main():
         run_calibration(args, rank, world, local_rank)
     elif args.workload == "prefill":
         run_prefill(args, rank, world, local_rank)
+    elif args.workload == "window_serving":
+        run_window(args, rank, world, local_rank)
     else:
         run_ours(args, rank, world, local_rank, cid=STEP_WORKLOADS[args.workload])
 

@@ -77,6 +77,8 @@ typedef enum { SQ_GATE_HEAD = 0 /* GDN */, SQ_GATE_KEY_CHANNEL = 1 /* KDA */ } s
 #define SQ_STATUS_SATURATED 2u  /* a row scale or pivot value saturated at +-65504 */
 #define SQ_STATUS_BAD_SLOT 4u   /* a slot id outside [0, n_slots) was skipped (o = 0) */
 #define SQ_STATUS_TIMEOUT 8u    /* a bounded device wait gave up (should never happen) */
+#define SQ_STATUS_WINDOW 16u    /* sq_window_step: a window record's count was outside [0, W);
+                                   the tile was skipped (o = 0, nothing written) */
 
 /* Shape of one layer's state pool. d_k == d_v == d, d in {32, 64, 128};
  * h_v % h_k == 0 (value head h reads key head h / (h_v / h_k)). */
@@ -175,6 +177,48 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
 sq_status sq_decode_step_host(sq_handle* h, void* pool, const float* q, const float* k, const float* v,
                               const float* beta, const float* g, float* o, const int32_t* slot_ids, int32_t B,
                               void* stream);
+
+/* Per-window variant of the decode step ("线性注意力每生成一个token都要搬状态，
+ * LeapQuant把它压到8位还不掉点" (wink.run), per-window quantization, the first
+ * of LeapQuant's three techniques): the packed state of a tile is frozen for
+ * a window of W tokens; every token's key k, update vector u and gate go to
+ * a high-precision buffer, the outputs come from the frozen state and the
+ * buffer together, and the state is requantized once when the window is
+ * full. The page gives no formula; the step computes, for a tile with n
+ * buffered tokens (this token is token n, its gate G_n; products of gates
+ * E_tau,i = G_{tau+1},i ... G_n,i, E_-1 over all n + 1 tokens):
+ *     S_ij = E_-1,i S0_ij + sum_{tau<n} E_tau,i k_tau,i u_tau,j   (S0 the frozen state)
+ *     u_j  = fp32(beta (v_j - sum_i S_ij k_i))
+ *     o_j  = fp32(sum_i (S_ij + k_i u_j) q_i)
+ * in fp64 (u and o rounded once), appends (k, u, G_n) as row n of the
+ * buffer, and at n + 1 = W requantizes S + k u^T (formed in fp64, scaled by
+ * fp32(1 / c_j), rounded to fp32) in place with the rules of sq_decode_step,
+ * then empties the buffer. Inside a window the pool is only read.
+ *   window_buf device, sq_window_buffer_bytes() bytes, caller-owned; record
+ *            of (slot s, value head h) at (s h_v + h) record_bytes:
+ *            [int32 count, 12 zero bytes][k: W x d fp32][u: W x d fp32]
+ *            [gates: W x gd fp32, zero-padded to a multiple of 4 floats],
+ *            gd = d (GATE_KEY_CHANNEL) or 1 (GATE_HEAD); row tau holds
+ *            buffered token tau. A slot whose state is (re)written by
+ *            sq_quantize_state or sq_prefill must have its records zeroed
+ *            (count 0) before its next window step. While count > 0 the
+ *            pool holds the state from before the buffered tokens.
+ *   W        window length, 1 <= W <= 64 (W = 1 is per-token
+ *            requantization, with fp64 instead of fp32 arithmetic); the
+ *            same W for every call on one buffer.
+ *   q .. o, slot_ids, B: as sq_decode_step (slot ids distinct).
+ * A count outside [0, W) skips the tile (o = 0, SQ_STATUS_WINDOW). Returns
+ * SQ_ERR_INVALID_ARG for an FP32 pool, W out of range, or a W whose
+ * working set does not fit in shared memory. */
+sq_status sq_window_step(sq_handle* h, void* pool, void* window_buf, int32_t W, const float* q, const float* k,
+                         const float* v, const float* beta, const float* g, float* o, const int32_t* slot_ids,
+                         int32_t B, void* stream);
+
+/* Plumbing (no passage). Sizes of the window buffer of sq_window_step for
+ * windows of W tokens: bytes of one (slot, head) record and of the whole
+ * buffer (n_slots h_v records). Returns SQ_ERR_INVALID_ARG for W outside
+ * [1, 64]. */
+sq_status sq_window_buffer_bytes(const sq_handle* h, int32_t W, uint64_t* record_bytes, uint64_t* buffer_bytes);
 
 /* Expand B pool slots to fp32 S [B, h_v, d, d] (device): S_ij = (q r) c_j for
  * quantized rows and h c_j for pivot rows. Skipped (bad) slots give 0. */

@@ -30,6 +30,7 @@ SQ_STATUS_NAN = 1
 SQ_STATUS_SATURATED = 2
 SQ_STATUS_BAD_SLOT = 4
 SQ_STATUS_TIMEOUT = 8
+SQ_STATUS_WINDOW = 16
 
 SQ_NOALLOC_MAX_HEADS = 64
 
@@ -109,10 +110,12 @@ def lib() -> ctypes.CDLL:
     L.sq_calib_add_tokens.argtypes = [P, P, P, I32, P]
     L.sq_calib_finish.argtypes = [P, ctypes.POINTER(CalibBudget), ctypes.POINTER(CalibOut), P]
     L.sq_calib_free.argtypes = [P]
+    L.sq_window_step.argtypes = [P, P, P, I32, P, P, P, P, P, P, P, I32, P]
+    L.sq_window_buffer_bytes.argtypes = [P, I32, ctypes.POINTER(U64), ctypes.POINTER(U64)]
     for name in ("sq_state_alloc", "sq_state_free", "sq_quantize_state", "sq_decode_step",
                  "sq_dequantize_state", "sq_state_bytes", "sq_head_layout", "sq_get_status",
                  "sq_prefill", "sq_decode_step_host", "sq_calib_allocate", "sq_calib_begin", "sq_calib_add_states", "sq_calib_add_tokens", "sq_calib_finish",
-                 "sq_calib_free"):
+                 "sq_calib_free", "sq_window_step", "sq_window_buffer_bytes"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -154,6 +157,16 @@ def sq_decode_step(h, pool, q, k, v, beta, g, o, slot_ids, B, stream) -> None:
 
 def sq_decode_step_host(h, pool, q, k, v, beta, g, o, slot_ids, B, stream) -> None:
     check(lib().sq_decode_step_host(h, pool, q, k, v, beta, g, o, slot_ids, B, stream))
+
+
+def sq_window_step(h, pool, wbuf, W, q, k, v, beta, g, o, slot_ids, B, stream) -> None:
+    check(lib().sq_window_step(h, pool, wbuf, W, q, k, v, beta, g, o, slot_ids, B, stream))
+
+
+def sq_window_buffer_bytes(h, W: int):
+    rb, tb = ctypes.c_uint64(), ctypes.c_uint64()
+    check(lib().sq_window_buffer_bytes(h, W, ctypes.byref(rb), ctypes.byref(tb)))
+    return rb.value, tb.value
 
 
 def sq_prefill(h, pool, S0, q, k, v, beta, g, o, S_out, lengths, slot_ids, B, L, stream) -> None:

@@ -15,6 +15,7 @@
 #include "sq_kernels.cuh"
 #include "sq_prefill.cuh"
 #include "sq_step.cuh"
+#include "sq_window.cuh"
 
 namespace sqi {
 
@@ -103,6 +104,9 @@ struct sq_handle {
   HostStage host_stage[2];
   cudaStream_t copy_stream = nullptr;
   uint64_t host_calls = 0;
+  // sq_window_step: launch plan of the last window length used
+  int win_W = 0, win_grid = 0;
+  uint32_t win_smem = 0;
 };
 
 namespace {
@@ -152,6 +156,7 @@ cudaError_t allow_all(int max_smem) {
   if (e == cudaSuccess) e = allow_max_smem(sqk::k_decode_step_fp32<D>, max_smem);
   if (e == cudaSuccess) e = allow_max_smem(sqk::k_quantize<D>, max_smem);
   if (e == cudaSuccess) e = allow_max_smem(sqk::k_dequantize<D>, max_smem);
+  if (e == cudaSuccess) e = allow_max_smem(sqk::k_window_step<D>, max_smem);
   return e;
 }
 
@@ -323,6 +328,41 @@ sq_status launch_step(sq_handle* h, void* pool, const float* q, const float* k, 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "launching the decode step");
   h->launches++;
+  return SQ_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------- per-window variant
+namespace {
+
+constexpr int kMaxWindow = 64;
+
+uint64_t window_record_bytes(int d, int gate, int W) {
+  const uint64_t gd = gate == SQ_GATE_KEY_CHANNEL ? (uint64_t)d : 1u;
+  return 16u + 4u * (2u * (uint64_t)W * d + round_up((uint64_t)W * gd, 4));
+}
+
+template <int D>
+sq_status window_plan(sq_handle* h, int W) {
+  const int gd = h->desc.gate == SQ_GATE_KEY_CHANNEL ? D : 1;
+  const sqk::WLay L = sqk::window_layout(D, W, gd);
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, sqk::k_window_step<D>);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+  if ((size_t)L.total + fa.sharedSizeBytes > (size_t)optin)
+    return fail(SQ_ERR_INVALID_ARG, "window of %d tokens needs %u bytes of shared memory per CTA (device limit %d)", W,
+                L.total + (unsigned)fa.sharedSizeBytes, optin);
+  int blocks = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, sqk::k_window_step<D>, sqk::WGeo<D>::NT, L.total);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (blocks < 1) return fail(SQ_ERR_INVALID_ARG, "window of %d tokens does not fit on an SM", W);
+  h->win_W = W;
+  h->win_smem = L.total;
+  h->win_grid = blocks * h->num_sms;
   return SQ_OK;
 }
 
@@ -600,6 +640,65 @@ sq_status sq_decode_step(sq_handle* h, void* pool, const float* q, const float* 
   return launch_step(h, pool, q, k, v, beta, g, o, slot_ids, B, stream);
 }
 
+
+
+sq_status sq_window_buffer_bytes(const sq_handle* h, int32_t W, uint64_t* record_bytes, uint64_t* buffer_bytes) {
+  g_last_error.clear();
+  if (!h || !record_bytes || !buffer_bytes) return fail(SQ_ERR_INVALID_ARG, "NULL argument");
+  if (W < 1 || W > kMaxWindow) return fail(SQ_ERR_INVALID_ARG, "W must be in [1, %d] (got %d)", kMaxWindow, W);
+  *record_bytes = window_record_bytes(h->d, h->desc.gate, W);
+  *buffer_bytes = *record_bytes * (uint64_t)h->desc.n_slots * (uint64_t)h->desc.h_v;
+  return SQ_OK;
+}
+
+sq_status sq_window_step(sq_handle* h, void* pool, void* window_buf, int32_t W, const float* q, const float* k,
+                         const float* v, const float* beta, const float* g, float* o, const int32_t* slot_ids,
+                         int32_t B, void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(SQ_ERR_INVALID_ARG, "NULL handle");
+  if (h->desc.fmt != SQ_FMT_PACKED) return fail(SQ_ERR_INVALID_ARG, "the window step needs a packed pool");
+  if (W < 1 || W > kMaxWindow) return fail(SQ_ERR_INVALID_ARG, "W must be in [1, %d] (got %d)", kMaxWindow, W);
+  if (B < 0) return fail(SQ_ERR_INVALID_ARG, "B must be >= 0 (got %d)", B);
+  if (B == 0) return SQ_OK;
+  if ((int64_t)B * h->desc.h_v > (int64_t)INT32_MAX / 2) return fail(SQ_ERR_INVALID_ARG, "B too large");
+  SQ_CHECK_PTR(pool, "pool");
+  SQ_CHECK_PTR(window_buf, "window_buf");
+  SQ_CHECK_PTR(q, "q");
+  SQ_CHECK_PTR(k, "k");
+  SQ_CHECK_PTR(v, "v");
+  SQ_CHECK_PTR(o, "o");
+  if (!beta) return fail(SQ_ERR_INVALID_ARG, "beta is NULL");
+  if (!g) return fail(SQ_ERR_INVALID_ARG, "g is NULL");
+  if (h->desc.gate == SQ_GATE_KEY_CHANNEL && !aligned16(g)) return fail(SQ_ERR_INVALID_ARG, "g is not 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(beta) & 3u) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(SQ_ERR_INVALID_ARG, "beta/g not 4-byte aligned");
+  if (slot_ids && (reinterpret_cast<uintptr_t>(slot_ids) & 3u)) return fail(SQ_ERR_INVALID_ARG, "slot_ids misaligned");
+  if (h->win_W != W) {
+    sq_status s = h->d == 128 ? window_plan<128>(h, W) : h->d == 64 ? window_plan<64>(h, W) : window_plan<32>(h, W);
+    if (s != SQ_OK) return s;
+  }
+  sqk::WindowArgs a{};
+  a.pool = static_cast<uint8_t*>(pool);
+  a.wbuf = static_cast<uint8_t*>(window_buf);
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.g = g; a.o = o;
+  a.slots = slot_ids;
+  a.B = B; a.h_v = h->desc.h_v; a.h_k = h->desc.h_k; a.n_slots = h->desc.n_slots; a.gate_kind = h->desc.gate;
+  a.W = W;
+  a.slot_bytes = h->slot_bytes;
+  a.wait_ns = h->wait_ns;
+  a.wrec_bytes = (uint32_t)window_record_bytes(h->d, h->desc.gate, W);
+  a.t = h->tables;
+  const int n_tiles = B * h->desc.h_v;
+  const int grid = n_tiles < h->win_grid ? n_tiles : h->win_grid;
+  cudaStream_t st = as_stream(stream);
+  if (h->d == 128) sqk::k_window_step<128><<<grid, sqk::WGeo<128>::NT, h->win_smem, st>>>(a);
+  else if (h->d == 64) sqk::k_window_step<64><<<grid, sqk::WGeo<64>::NT, h->win_smem, st>>>(a);
+  else sqk::k_window_step<32><<<grid, sqk::WGeo<32>::NT, h->win_smem, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launching the window step");
+  h->launches++;
+  return SQ_OK;
+}
 
 sq_status sq_decode_step_host(sq_handle* h, void* pool, const float* q, const float* k, const float* v,
                               const float* beta, const float* g, float* o, const int32_t* slot_ids, int32_t B,

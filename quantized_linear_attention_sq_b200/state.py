@@ -124,6 +124,30 @@ class StatePool:
                             _ptr(g, torch.float32, "g", gn), _ptr(o, torch.float32, "o", B * hv * d),
                             _ptr(slot_ids, torch.int32, "slot_ids", B), B, _stream(stream))
 
+    def window_buffer_bytes(self, W: int):
+        """(bytes of one (slot, head) window record, bytes of the whole buffer)."""
+        return _abi.sq_window_buffer_bytes(self._h, int(W))
+
+    def new_window_buffer(self, W: int) -> torch.Tensor:
+        """A zeroed window buffer (every count 0) for windows of W tokens."""
+        return torch.zeros(self.window_buffer_bytes(W)[1], dtype=torch.uint8, device=self.device)
+
+    def window_step(self, pool, wbuf, W, q, k, v, beta, g, o, slot_ids=None, stream=None):
+        """One token of the per-window variant (sq_window_step): the packed
+        state stays frozen while the window buffer collects the tokens'
+        updates; it is requantized when W tokens are buffered."""
+        B = q.shape[0]
+        d, hv, hk = self.d, self.h_v, self.h_k
+        gn = B * hv * (d if self.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1)
+        nb = self.window_buffer_bytes(W)[1]
+        if wbuf.numel() * wbuf.element_size() != nb:
+            raise ValueError(f"window buffer has {wbuf.numel() * wbuf.element_size()} bytes, expected {nb}")
+        _abi.sq_window_step(self._h, self._check_pool(pool), _ptr(wbuf, name="wbuf"), int(W),
+                            _ptr(q, torch.float32, "q", B * hk * d), _ptr(k, torch.float32, "k", B * hk * d),
+                            _ptr(v, torch.float32, "v", B * hv * d), _ptr(beta, torch.float32, "beta", B * hv),
+                            _ptr(g, torch.float32, "g", gn), _ptr(o, torch.float32, "o", B * hv * d),
+                            _ptr(slot_ids, torch.int32, "slot_ids", B), B, _stream(stream))
+
     def decode_step_host(self, pool, q, k, v, beta, g, o, slot_ids=None, stream=None):
         """The decode step with q, k, v, beta, g, slot_ids and o as CPU tensors
         (page-locked for overlapped copies; o page-locked is written by the

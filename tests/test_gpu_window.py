@@ -1,0 +1,166 @@
+"""GPU parity of the per-window variant (sq_window_step) against the oracle.
+
+Per-window quantization ("线性注意力每生成一个token都要搬状态，LeapQuant把它压到
+8位还不掉点" (wink.run), first technique). Both sides start from the same
+quantized bytes and empty window buffers and take the same tokens; after
+every token the outputs, the window buffers and the pools are compared:
+
+- o within the step's tolerance (relative L2);
+- window records: counts, buffered keys and gates identical; buffered u
+  identical except where the fp64 sums of the two sides (different orders)
+  straddle an fp32 rounding boundary: at most one fp32 ulp, rarely;
+- pools: identical inside a window (the state is frozen) and, after the
+  window's requantization, codes identical up to the step's rare 1-LSB flips
+  (the requantized state is formed in the same order of fp64 operations on
+  both sides, so it differs only where the buffered u did).
+Where anything differs the GPU continues from the oracle's bytes (teacher
+forcing)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_linear_attention_sq_b200 import _abi, synth
+from tests.gpu_util import (THREADS, Stats, compare_slots, gpu_pool_for, oracle_warm_state, slot_bytes, to_dev)
+from tests.helpers import oracle_for, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+U_ULP_RATE = 1e-3  # buffered u values allowed to differ (by one ulp)
+
+
+def _wrec_view(buf: np.ndarray, n_rec: int, rb: int):
+    return buf.reshape(n_rec, rb)
+
+
+def compare_windows(ref: np.ndarray, got: np.ndarray, rb: int, W: int, d: int, gd: int, counters: dict):
+    R, G = _wrec_view(ref, -1, rb), _wrec_view(got, -1, rb)
+    assert np.array_equal(R[:, :16], G[:, :16]), "window counts differ"
+    k0, k1 = 16, 16 + 4 * W * d
+    u1 = k1 + 4 * W * d
+    assert np.array_equal(R[:, k0:k1], G[:, k0:k1]), "buffered keys differ"
+    assert np.array_equal(R[:, u1:], G[:, u1:]), "buffered gates differ"
+    ur = R[:, k1:u1].copy().view(np.float32)
+    ug = G[:, k1:u1].copy().view(np.float32)
+    diff = ur != ug
+    counters["u_entries"] += ur.size
+    if diff.any():
+        a, b = ur[diff].astype(np.float64), ug[diff].astype(np.float64)
+        ulp = np.spacing(np.maximum(np.abs(a), np.abs(b)).astype(np.float32)).astype(np.float64)
+        assert (np.abs(a - b) <= ulp).all(), "a buffered u differs by more than one ulp"
+        counters["u_diff"] += int(diff.sum())
+    return bool(diff.any())
+
+
+def run_window_parity(cid: int, W: int, steps: int, check_requests=None, batch=None):
+    w = synth.workload(cid, batch=batch)
+    c = w.cfg
+    B = w.B
+    reqs = list(range(B)) if check_requests is None else list(check_requests)
+    sel = np.asarray(reqs)
+    o_ = oracle_for(oracle, w, n_slots=len(reqs))
+    sp = gpu_pool_for(w, B)
+    rb, _ = sp.window_buffer_bytes(W)
+    assert rb == o_.window_record_bytes(W)
+    gd = c.d if c.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1
+    # initial state: the checked requests start from the oracle's fp32 state
+    S_ref = oracle_warm_state(w, reqs)
+    S_all = torch.from_numpy(w.initial_state()).cuda()
+    S_all.index_copy_(0, torch.as_tensor(reqs, device="cuda"), torch.from_numpy(S_ref).cuda())
+    pool_ref = o_.new_pool()
+    o_.quantize(pool_ref, S_ref)
+    pool = sp.new_pool()
+    sp.quantize_state(pool, S_all)
+    del S_all
+    wref = o_.new_window_buffer(W)
+    wbuf = sp.new_window_buffer(W)
+    gslots = sel.astype(np.int32)
+    assert np.array_equal(slot_bytes(pool, sp, gslots), pool_ref)
+    o_dev = torch.empty((B, c.h_v, c.d), device="cuda")
+    stats = Stats()
+    counters = {"u_entries": 0, "u_diff": 0}
+    st_all = 0
+    idx = torch.as_tensor(gslots, device="cuda", dtype=torch.long)
+    for t in range(steps):
+        q, k, v, beta, g = w.step_inputs(t)
+        sp.window_step(pool, wbuf, W, *to_dev(q, k, v, beta, g), o_dev)
+        o_ref, st_ref = o_.window_step(pool_ref, wref, W, q[sel], k[sel], v[sel], beta[sel], g[sel],
+                                       threads=THREADS)
+        st_all |= st_ref
+        o_got = o_dev.cpu().numpy()[sel]
+        stats.worst_o = max(stats.worst_o, rel_l2(o_got, o_ref))
+        got_w = wbuf.view(B * c.h_v, rb).index_select(0, (idx[:, None] * c.h_v + torch.arange(
+            c.h_v, device="cuda")[None]).reshape(-1)).cpu().numpy().reshape(-1)
+        u_diff = compare_windows(wref, got_w, rb, W, c.d, gd, counters)
+        got = slot_bytes(pool, sp, gslots)
+        f0 = stats.flips + stats.r_flips
+        compare_slots(o_, pool_ref, got, stats)
+        stats.steps += 1
+        if u_diff or stats.flips + stats.r_flips != f0:
+            pv = pool.view(-1, sp.slot_bytes)
+            pv[idx] = torch.from_numpy(pool_ref.reshape(len(reqs), -1)).cuda()
+            wv = wbuf.view(B, -1)
+            wv[idx] = torch.from_numpy(wref.reshape(len(reqs), -1)).cuda()
+    st_gpu = sp.get_status()
+    if len(reqs) == B:
+        assert st_gpu == st_all, (st_gpu, st_all)
+    sp.close()
+    return stats, counters
+
+
+@pytest.mark.parametrize("cid,W,steps", [(0, 4, 11), (0, 16, 35), (0, 1, 5)])
+def test_window_plumbing(cid, W, steps):
+    stats, cnt = run_window_parity(cid, W, steps)
+    print(stats, cnt)
+    stats.check()
+    assert cnt["u_diff"] <= U_ULP_RATE * cnt["u_entries"], cnt
+
+
+@pytest.mark.parametrize("cid", [1, 2])
+def test_window_layer(cid):
+    """GDN and KDA layers (mixed widths, pivots, outlier columns), W = 16,
+    over two windows and a bit."""
+    stats, cnt = run_window_parity(cid, 16, 35, check_requests=[0, 5, 17, 63])
+    print(stats, cnt)
+    stats.check()
+    assert cnt["u_diff"] <= U_ULP_RATE * cnt["u_entries"], cnt
+
+
+def test_window_serving_full_size():
+    """The GDN serving batch (512 requests x 32 heads) as the bench launches
+    it; sampled requests checked against the oracle through one window end."""
+    stats, cnt = run_window_parity(3, 16, 18, check_requests=[0, 1, 255, 511])
+    print(stats, cnt)
+    stats.check()
+    assert cnt["u_diff"] <= U_ULP_RATE * cnt["u_entries"], cnt
+
+
+def test_window_bad_count_and_slot():
+    """A window count outside [0, W) skips the tile (o = 0, status bit, the
+    pool and the buffer untouched); so does a slot id out of range."""
+    w = synth.workload(0)
+    c = w.cfg
+    sp = gpu_pool_for(w, 2)
+    W = 8
+    rb, nb = sp.window_buffer_bytes(W)
+    pool = sp.new_pool()
+    sp.quantize_state(pool, torch.from_numpy(np.repeat(w.initial_state(), 2, 0)).cuda())
+    wbuf = sp.new_window_buffer(W)
+    wbuf.view(-1, rb)[0, :4] = torch.tensor([W, 0, 0, 0], dtype=torch.uint8)  # slot 0, head 0: count W
+    pool0, w0 = pool.clone(), wbuf.clone()
+    q, k, v, beta, g = to_dev(*w.step_inputs(0))
+    o = torch.full((1, c.h_v, c.d), 7.0, device="cuda")
+    sp.get_status()
+    sp.window_step(pool, wbuf, W, q, k, v, beta, g, o, torch.tensor([0], dtype=torch.int32, device="cuda"))
+    assert sp.get_status() == _abi.SQ_STATUS_WINDOW
+    assert (o[0, 0] == 0).all() and (o[0, 1:] != 7.0).all()
+    assert torch.equal(wbuf.view(-1, rb)[0], w0.view(-1, rb)[0])
+    assert torch.equal(pool, pool0)  # inside a window the pool is only read
+    sp.window_step(pool, wbuf, W, q, k, v, beta, g, o, torch.tensor([5], dtype=torch.int32, device="cuda"))
+    assert sp.get_status() == _abi.SQ_STATUS_BAD_SLOT
+    assert (o == 0).all()
+    with pytest.raises(_abi.SQError):
+        sp.window_step(pool, wbuf, 0, q, k, v, beta, g, o)
+    with pytest.raises(_abi.SQError):
+        sp.window_step(pool, wbuf, 65, q, k, v, beta, g, o)
+    sp.close()
