@@ -639,8 +639,9 @@ uint32_t sqo_step_fp32(const sqo_desc *D, float *Spool, const float *q, const fl
  *   p_j = sum_i Sg_ij k_n,i ; u_n,j = fp32(beta (v_j - p_j))
  *   S_ij = Sg_ij + k_n,i u_n,j ; o_j = fp32(sum_i S_ij q_n,i)
  * then token n is appended (count n + 1), and when count reaches W the
- * state is requantized once, T'_ij = fp32(S_ij ic_j) with ic_j = fp32(1/c_j),
- * by the step's requantization (store_T), and count returns to 0.
+ * state is requantized once by the step's requantization (store_T) from
+ * its column-normalised form, summed in fp32 like the step's T' (below),
+ * and count returns to 0.
  * A slot id out of range skips the tile (o = 0, status bit). */
 static size_t window_gate_floats(const sqo_desc *D, int W) {
   size_t n = (size_t)W * (D->gate_kind == 0 ? 1 : (size_t)D->d);
@@ -709,11 +710,28 @@ static uint32_t window_tile(const sqo_desc *D, uint8_t *rec, uint8_t *wrec, int 
   }
   n += 1;
   if (n == W) {
-    for (int i = 0; i < d; i++)
+    /* The window's W tokens are all in the buffer (the current one last,
+     * with no gate after it). In the column-normalised units of the
+     * record, the state is the frozen term plus W rank-one terms:
+     *   T_ij = V_ij a_i + sum_tau e_tau,i w_tau,j
+     *   a_i = fp32(D_-1,i M_i), e_tau,i = fp32(D_tau,i k_tau,i) (D = 1 for the
+     *   current token), w_tau,j = fp32(u_tau,j ic_j), as the step's w = u / c;
+     * summed in fp32 the way the step forms T': t = fmaf(e, w, t) over the
+     * tokens in order from t = 0, then T = fmaf(V, a, t). */
+    for (int i = 0; i < d; i++) {
+      const float a = (float)(Dg[i] * (double)M[i]);
       for (int j = 0; j < d; j++) {
-        float ic = 1.0f / c[j];
-        T[i * d + j] = (float)(S[i * d + j] * (double)ic);
+        const float ic = 1.0f / c[j];
+        float t = 0.0f;
+        for (int tau = 0; tau < W; tau++) {
+          const double Dt = tau < W - 1 ? Dg[(size_t)(tau + 1) * d + i] : 1.0;
+          const float e = (float)(Dt * (double)kb[(size_t)tau * d + i]);
+          const float w = ub[(size_t)tau * d + j] * ic;
+          t = fmaf(e, w, t);
+        }
+        T[i * d + j] = fmaf(V[i * d + j], a, t);
       }
+    }
     st |= store_T(D, h, rec, T);
     n = 0;
   }
