@@ -20,15 +20,17 @@
 //   o_j = sum_i (S_ij + k_i u_j) q_i
 //       = c_j sum_i V_ij b_i + sum_tau gamma_tau u_tau,j + (k . q) u_j,
 //         b_i = E_-1,i M_i q_i,  gamma_tau = sum_i E_tau,i k_tau,i q_i
-// so a token reads the packed codes once and forms two column sums of them
-// (p in fp64, o in fp32), reads the buffer's n rows, appends its own row, and
-// writes nothing of the state. When the window is full, the state
-// S_ij + k_i u_j is formed in fp64 one rounded operation at a time, in the
-// order of the definition (E_-1,i ((V_ij M_i) c_j), then the buffered terms
-// (E_tau,i k_tau,i) u_tau,j in token order, then k_i u_j), scaled by
-// fp32(1/c_j), rounded to fp32 and requantized in place by the step's rules
-// (row scales from the row maximum and the clip ratio, round-up to fp16,
-// codes rounded to nearest even).
+// so a token reads the packed codes once and forms two fp64 column sums of
+// them, reads the buffer's n rows, appends its own row, and writes nothing
+// of the state. When the window is full the state is formed in the record's
+// column-normalised units and in fp32, the way the step forms T':
+//   T_ij = fmaf(V_ij, a_i, t_ij),  t_ij = fmaf(e_tau,i, w_tau,j, t_ij) over the
+//   W tokens in order from t = 0,  a_i = fp32(E_-1,i M_i),
+//   e_tau,i = fp32(E_tau,i k_tau,i) (E = 1 for the last token),
+//   w_tau,j = fp32(u_tau,j fp32(1/c_j))
+// (a rank-W update of the frozen state), and requantized in place by the
+// step's rules (row scales from the row maximum and the clip ratio,
+// round-up to fp16, codes rounded to nearest even).
 //
 // Work distribution. Persistent CTAs: four consumer warps in the packed
 // step's thread map (PGeo: a thread owns 16 columns of RPT key rows) and one
@@ -81,13 +83,15 @@ struct WHdr {
 
 // Stage layout (bytes): [hdr 64][q][k][v][g][col][icol] (fp32, d each)
 // [row_off u16 d][row_code d][row_perm d][k rows fp32 (W-1) d][u rows fp32 (W-1) d]
-// [gates fp32 (W-1) gd, padded to 16 B], padded to 128 B. Then, after both
-// stages, the work area: [S^T k partials fp64 NG d][o partials fp32 NG d]
-// [E k products fp64 (W-1) d][a fp64 d][E_-1 fp64 d][b fp32 d][M fp32 d]
-// [u fp32 d][alpha, gamma fp64 W each, k.q, pad].
+// [gates fp32 (W-1) gd, padded to 16 B], padded to 128 B. At a window's end
+// the k rows are replaced by e rows and the u rows by w rows. Then, after
+// both stages, the work area: [S^T k partials fp64 NW d][S^T q partials fp64
+// NW d][E k products fp64 (W-1) d][a][b][k][q][E_-1] (fp64 d each)
+// [M][u or w][a][e of the current token] (fp32 d each)[alpha, gamma fp64 W
+// each, k.q, pad].
 struct WLay {
   uint32_t q, k, v, g, col, icol, roff, rcode, rperm, kb, ub, gb, stage;
-  uint32_t redp, redo, ek, a, d0, b, m, un, ag, total;
+  uint32_t redp, redo, ek, a, b, kd, qd, d0, m, un, af, ecur, ag, total;
 };
 __host__ __device__ inline uint32_t wround(uint32_t x, uint32_t m) { return (x + m - 1) / m * m; }
 __host__ __device__ inline WLay window_layout(int D, int W, int gd) {
@@ -106,18 +110,50 @@ __host__ __device__ inline WLay window_layout(int D, int W, int gd) {
   L.ub = L.kb + 4 * w1 * d;
   L.gb = L.ub + 4 * w1 * d;
   L.stage = wround(L.gb + 4 * wround(w1 * (uint32_t)gd, 4), 128);
-  const uint32_t ng = 16;
+  const uint32_t nw = (uint32_t)D / 32;  // consumer warps (PGeo: D threads)
   L.redp = 2 * L.stage;
-  L.redo = L.redp + 8 * ng * d;
-  L.ek = L.redo + 4 * ng * d;
+  L.redo = L.redp + 8 * nw * d;
+  L.ek = L.redo + 8 * nw * d;
   L.a = L.ek + 8 * (w1 > 0 ? w1 : 1) * d;
-  L.d0 = L.a + 8 * d;
-  L.b = L.d0 + 8 * d;
-  L.m = L.b + 4 * d;
+  L.b = L.a + 8 * d;
+  L.kd = L.b + 8 * d;
+  L.qd = L.kd + 8 * d;
+  L.d0 = L.qd + 8 * d;
+  L.m = L.d0 + 8 * d;
   L.un = L.m + 4 * d;
-  L.ag = L.un + 4 * d;
+  L.af = L.un + 4 * d;
+  L.ecur = L.af + 4 * d;
+  L.ag = L.ecur + 4 * d;
   L.total = wround(L.ag + 8 * (2 * (uint32_t)W + 2), 128);
   return L;
+}
+
+// Column sums of the 16 fp64 partials of every thread: the RPW row groups of
+// a warp are added by shuffles, then the warp's lanes of row group 0 deposit
+// (16-byte pieces rotated by cc against bank conflicts) and thread j adds
+// the NW warps' values of column j.
+template <int D>
+__device__ __forceinline__ void wdeposit(double* red, int warp, int lane, int cc, double (&acc)[16]) {
+  using G = PGeo<D>;
+#pragma unroll
+  for (int o = G::LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+  if (lane < G::LPR) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      *reinterpret_cast<double2*>(red + warp * D + 16 * cc + 2 * (p ^ (cc & 7))) =
+          make_double2(acc[2 * p], acc[2 * p + 1]);
+  }
+}
+template <int D>
+__device__ __forceinline__ double wtotal(const double* red, int j) {
+  const int cj = j >> 4, e = j & 15;
+  const int off = 16 * cj + 2 * ((e >> 1) ^ (cj & 7)) + (e & 1);
+  double t = 0.0;
+#pragma unroll
+  for (int w = 0; w < PGeo<D>::NW; ++w) t += red[w * D + off];
+  return t;
 }
 
 template <int D>
@@ -127,6 +163,32 @@ struct WGeo {
 };
 
 __device__ __forceinline__ void consumer_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
+
+// Bounded wait on an mbarrier phase that suspends the thread in the
+// hardware until the phase completes (or a 20 us hint runs out) instead of
+// polling, so that a waiting warp takes no issue slots from the others.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_suspend(uint64_t* bar, uint32_t parity, uint64_t max_ns) {
+  if (mbar_try_wait_suspend(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    uint64_t t1;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+    if (t1 - t0 > max_ns) return false;
+  }
+}
 
 // The producer's view of one tile (loads issued one tile ahead of use).
 struct WScal {
@@ -209,46 +271,55 @@ __device__ __forceinline__ void wissue(const WindowArgs& a, const WLay& L, uint8
   bulk_prefetch_l2(rec, x.rec_bytes);
 }
 
+// Position of column j in a rotated w row: the four 4-column pieces of each
+// 16-column chunk cj are rotated by cj / 2, so that chunk cc's piece p is at
+// 4 ((p + cc / 2) mod 4).
+__device__ __forceinline__ int wswz(int j) {
+  const int cj = j >> 4, e = j & 15;
+  return 16 * cj + 4 * (((e >> 2) + (cj >> 1)) & 3) + (e & 3);
+}
+
 // Pointers into the work area.
 struct WWork {
   double* redp;
-  float* redo;
+  double* redo;
   double* ek;
   double* a;
+  double* b;
+  double* kd;
+  double* qd;
   double* d0;
-  float* b;
   float* m;
   float* un;
+  float* af;
+  float* ecur;
   double* ag;
 };
 
-// One row's contribution to the two column sums: 16 fp64 views (high words,
-// see field_hi) times a_i into accP, the 16 codes (exact, from the same
-// words read as floats) times b_i into accO.
+// One row's contribution to the two column sums: the 16 codes as fp64 views
+// (high words: 2^E + field, see field_hi), times a_i into accP and b_i into
+// accO; the views' offset 2^E + 2^(b-1) is taken off once per row (offP, offO).
 template <int B>
-__device__ __forceinline__ void wrow_q(const uint32_t* w, double ai, float bi, double (&accP)[16], float2 (&accO)[8]) {
-  using F = FieldPos<B>;
-  uint32_t xh[16];
+__device__ __forceinline__ void wrow_q(const uint32_t* w, double ai, double bi, double (&accP)[16],
+                                       double (&accO)[16]) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j) xh[j] = field_hi<B>(w, j);
-#pragma unroll
-  for (int j = 0; j < 16; ++j) accP[j] = fma(__hiloint2double((int)xh[j], 0), ai, accP[j]);
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const float2 x = make_float2(__uint_as_float(xh[2 * p]), __uint_as_float(xh[2 * p + 1]));
-    const float2 qv = __ffma2_rn(x, f2(F::K), f2(-F::C));
-    accO[p] = __ffma2_rn(qv, f2(bi), accO[p]);
+  for (int j = 0; j < 16; ++j) {
+    const double x = __hiloint2double((int)field_hi<B>(w, j), 0);
+    accP[j] = fma(x, ai, accP[j]);
+    accO[j] = fma(x, bi, accO[j]);
   }
 }
 // A pivot row: 16 fp16 values.
-__device__ __forceinline__ void wrow_pivot(const uint32_t* w, double ai, float bi, double (&accP)[16],
-                                           float2 (&accO)[8]) {
+__device__ __forceinline__ void wrow_pivot(const uint32_t* w, double ai, double bi, double (&accP)[16],
+                                           double (&accO)[16]) {
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
-    accP[2 * p] = fma((double)x.x, ai, accP[2 * p]);
-    accP[2 * p + 1] = fma((double)x.y, ai, accP[2 * p + 1]);
-    accO[p] = __ffma2_rn(x, f2(bi), accO[p]);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
+    const double x0 = (double)f.x, x1 = (double)f.y;
+    accP[2 * p] = fma(x0, ai, accP[2 * p]);
+    accP[2 * p + 1] = fma(x1, ai, accP[2 * p + 1]);
+    accO[2 * p] = fma(x0, bi, accO[2 * p]);
+    accO[2 * p + 1] = fma(x1, bi, accO[2 * p + 1]);
   }
 }
 // The b/2 words (quantized row) or 8 words (pivot row) of chunk cc, read from
@@ -263,23 +334,29 @@ __device__ __forceinline__ void wload_words(const uint8_t* row, int code, int cc
 }
 
 // The frozen pass of a head whose rows all have width KC (ROW_PIVOT: all
-// pivot): every row's chunk is loaded first (one round trip), then used.
+// pivot): the chunks of all of the thread's rows are loaded first (pivot
+// heads: four rows at a time), then used.
 template <int D, int KC>
 __device__ __forceinline__ void wfrozen_uniform(const uint8_t* rec, const WWork& w, int rg, int cc,
-                                                double (&accP)[16], float2 (&accO)[8]) {
+                                                double (&accP)[16], double (&accO)[16]) {
   using G = PGeo<D>;
   constexpr int NWD = KC == ROW_PIVOT ? 8 : KC / 2;
   constexpr uint32_t rb = KC == ROW_PIVOT ? 2u * D : (uint32_t)(D * KC / 8);
-  // rows in batches of at most 16 words of codes per thread
-  constexpr int RB = G::RPT * NWD <= 16 ? G::RPT : (NWD <= 4 ? 4 : 2);
+  constexpr int RB = NWD <= 4 ? G::RPT : (G::RPT < 4 ? G::RPT : 4);
   static_assert(G::RPT % RB == 0, "row batches");
-  double off = 0.0;
+  double offP = 0.0, offO = 0.0;
   if constexpr (KC != ROW_PIVOT) {
 #pragma unroll
-    for (int r = 0; r < G::RPT; ++r) off += code_offset(KC) * w.a[r * G::NG + rg];
+    for (int r = 0; r < G::RPT; ++r) {
+      offP += code_offset(KC) * w.a[r * G::NG + rg];
+      offO += code_offset(KC) * w.b[r * G::NG + rg];
+    }
   }
 #pragma unroll
-  for (int j = 0; j < 16; ++j) accP[j] = -off;
+  for (int j = 0; j < 16; ++j) {
+    accP[j] = -offP;
+    accO[j] = -offO;
+  }
 #pragma unroll
   for (int r0 = 0; r0 < G::RPT; r0 += RB) {
     uint32_t wd[RB][NWD];
@@ -304,17 +381,23 @@ __device__ __forceinline__ void wfrozen_uniform(const uint8_t* rec, const WWork&
 template <int D>
 __device__ __forceinline__ void wfrozen_mixed(const uint8_t* rec, const uint16_t* roff, const uint8_t* rcode,
                                               const uint8_t* rperm, uint32_t bytes, const WWork& w, int rg, int cc,
-                                              double (&accP)[16], float2 (&accO)[8]) {
+                                              double (&accP)[16], double (&accO)[16]) {
   using G = PGeo<D>;
-  double off = 0.0;
+  double offP = 0.0, offO = 0.0;
 #pragma unroll 1
   for (int r = 0; r < G::RPT; ++r) {
     const int i = rperm[r * G::NG + rg] & (D - 1);
     const int code = rcode[i];
-    if (code != ROW_PIVOT) off += code_offset(code) * w.a[i];
+    if (code != ROW_PIVOT) {
+      offP += code_offset(code) * w.a[i];
+      offO += code_offset(code) * w.b[i];
+    }
   }
 #pragma unroll
-  for (int j = 0; j < 16; ++j) accP[j] = -off;
+  for (int j = 0; j < 16; ++j) {
+    accP[j] = -offP;
+    accO[j] = -offO;
+  }
   uint32_t nxt[8];
   int inext = rperm[rg] & (D - 1);
   int cnext = rcode[inext];
@@ -331,7 +414,7 @@ __device__ __forceinline__ void wfrozen_mixed(const uint8_t* rec, const uint16_t
       wload_words(rec + min((uint32_t)roff[inext], bytes), cnext, cc, nxt);
     }
     const double ai = w.a[i];
-    const float bi = w.b[i];
+    const double bi = w.b[i];
     switch (code) {
       case 8: wrow_q<8>(cur, ai, bi, accP, accO); break;
       case 6: wrow_q<6>(cur, ai, bi, accP, accO); break;
@@ -344,7 +427,7 @@ __device__ __forceinline__ void wfrozen_mixed(const uint8_t* rec, const uint16_t
 
 // One tile. Returns status bits.
 template <int D, int KC>
-__device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, const uint8_t* stg, const WHdr* hd,
+__device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, uint8_t* stg, const WHdr* hd,
                                           const WWork& w, int rg, int cc) {
   using G = PGeo<D>;
   constexpr int NC = WGeo<D>::NC;
@@ -366,7 +449,7 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
   const uint8_t* rcode = stg + L.rcode;
   const uint8_t* rperm = stg + L.rperm;
   const float* kb = reinterpret_cast<const float*>(stg + L.kb);
-  const float* ub = reinterpret_cast<const float*>(stg + L.ub);
+  float* ub = reinterpret_cast<float*>(stg + L.ub);  // turned into w rows at a window's end
   const float* gb = reinterpret_cast<const float*>(stg + L.gb);
   uint32_t st = 0;
 
@@ -382,8 +465,11 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
     const int code = KC ? KC : rcode[i];
     const float M = code == ROW_PIVOT ? 1.0f : __half2float(reinterpret_cast<const __half*>(rec)[i]);
     const double DM = __dmul_rn(acc, (double)M);
-    w.a[i] = __dmul_rn(DM, (double)sk[i]);
-    w.b[i] = __double2float_rn(__dmul_rn(DM, (double)sq[i]));
+    const double ki = (double)sk[i], qi = (double)sq[i];
+    w.a[i] = __dmul_rn(DM, ki);
+    w.b[i] = __dmul_rn(DM, qi);
+    w.kd[i] = ki;
+    w.qd[i] = qi;
     w.d0[i] = acc;
     w.m[i] = M;
   }
@@ -395,9 +481,10 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
     double sa = 0.0, sgm = 0.0;
 #pragma unroll
     for (int x = lane; x < D; x += 32) {
-      const double e = tau < n ? w.ek[tau * D + x] : (double)sk[x];
-      sa = fma(e, (double)sk[x], sa);
-      sgm = fma(e, (double)sq[x], sgm);
+      const double kx = w.kd[x];
+      const double e = tau < n ? w.ek[tau * D + x] : kx;
+      sa = fma(e, kx, sa);
+      sgm = fma(e, w.qd[x], sgm);
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -410,29 +497,26 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
     }
   }
 
-  // ---- frozen pass: column sums of the codes against a (fp64) and b (fp32)
+  // ---- frozen pass: column sums of the codes against a and b (fp64)
   {
-    double accP[16];
-    float2 accO[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) accO[p] = make_float2(0.0f, 0.0f);
+    double accP[16], accO[16];
     if constexpr (KC != 0)
       wfrozen_uniform<D, KC>(rec, w, rg, cc, accP, accO);
     else
       wfrozen_mixed<D>(rec, roff, rcode, rperm, hd->bytes, w, rg, cc, accP, accO);
-    pdeposit_f64<D>(w.redp, rg, cc, accP);
-    pdeposit_f32<D>(w.redo, rg, cc, accO);
+    wdeposit<D>(w.redp, warp, lane, cc, accP);
+    wdeposit<D>(w.redo, warp, lane, cc, accO);
   }
   consumer_sync(NC);  // partials, alpha, gamma complete
 
   // ---- per column j = tid: p, u, o; append token n to the window
   {
     const int j = tid;
-    const double Pt = ptotal_f64<D>(w.redp, j);
-    const float Ot = ptotal_f32<D>(w.redo, j);
+    const double Pt = wtotal<D>(w.redp, j);
+    const double Ot = wtotal<D>(w.redo, j);
     const double cj = (double)scol[j];
     double p = __dmul_rn(cj, Pt);
-    double oo = __dmul_rn(cj, (double)Ot);
+    double oo = __dmul_rn(cj, Ot);
 #pragma unroll 1
     for (int tau = 0; tau < n; ++tau) {
       const double u = (double)ub[tau * D + j];
@@ -453,32 +537,84 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
       wg[n * D + j] = sg[j];
     else if (j == 0)
       wg[n] = hd->g;
-    w.un[j] = un;
     if (n + 1 < W) {
       if (j == 0) *reinterpret_cast<int32_t*>(hd->wrec) = n + 1;
       return st;
     }
+    w.un[j] = __fmul_rn(un, sicol[j]);  // the current token's w
   }
 
-  // ---- end of the window: form the state in fp64, requantize in place
-  consumer_sync(NC);  // u complete
+  // ---- end of the window: T = V a + sum_tau e_tau w_tau in fp32, requantized
+  // in place (the record's column-normalised units; see the oracle's
+  // definition: t = fmaf(e, w, t) over the tokens in order, T = fmaf(V, a, t))
+  consumer_sync(NC);  // w of the current token is in
+  float* e = reinterpret_cast<float*>(stg + L.kb);  // [tau][row] over the buffered keys (used up)
+  {
+    const int i = tid;
+    for (int tau = 0; tau < n; ++tau) e[tau * D + i] = __double2float_rn(w.ek[tau * D + i]);
+    w.ecur[i] = sk[i];
+    w.af[i] = __double2float_rn(__dmul_rn(w.d0[i], (double)w.m[i]));
+    // as column j = i: the buffered u rows become w rows, each 16-column
+    // chunk stored rotated (wswz) so that the lanes of a row group read
+    // their chunks from different banks; the 16 columns of a chunk belong
+    // to 16 lanes of one warp, which read before any of them writes
+    const float icj = sicol[i];
+    const int si = wswz(i);
+    for (int tau = 0; tau < n; ++tau) {
+      const float x = __fmul_rn(ub[tau * D + i], icj);
+      __syncwarp();
+      ub[tau * D + si] = x;
+      __syncwarp();
+    }
+    const float xc = w.un[i];
+    __syncwarp();
+    w.un[si] = xc;
+  }
+  consumer_sync(NC);  // e, a, w complete
   const float* phi = a.t.phi + (size_t)h * D;
   constexpr bool DIRECT = KC == ROW_PIVOT;
 #pragma unroll 1
   for (int grp = 0; grp < G::RPT / G::QS; ++grp) {
-    float2 T[G::QS][8];
+    int rows[G::QS];
 #pragma unroll
     for (int u = 0; u < G::QS; ++u) {
       const int s = (grp * G::QS + u) * G::NG + rg;
-      const int i = KC ? s : (rperm[s] & (D - 1));
-      const int code = KC ? KC : rcode[i];
+      rows[u] = KC ? s : (rperm[s] & (D - 1));
+    }
+    float2 T[G::QS][8];
+#pragma unroll
+    for (int u = 0; u < G::QS; ++u)
+#pragma unroll
+      for (int p = 0; p < 8; ++p) T[u][p] = make_float2(0.0f, 0.0f);
+    // t += e_tau (x) w_tau for the buffered tokens, then the current one
+    auto add_token = [&](const float* wrow, const float* erow) {
+      float2 wv[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float4 x = *reinterpret_cast<const float4*>(wrow + 16 * cc + 4 * ((p + (cc >> 1)) & 3));
+        wv[2 * p] = make_float2(x.x, x.y);
+        wv[2 * p + 1] = make_float2(x.z, x.w);
+      }
+#pragma unroll
+      for (int u = 0; u < G::QS; ++u) {
+        const float2 ev = f2(erow[rows[u]]);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) T[u][p] = __ffma2_rn(ev, wv[p], T[u][p]);
+      }
+    };
+#pragma unroll 2
+    for (int tau = 0; tau < n; ++tau) add_token(ub + tau * D, e + tau * D);
+    add_token(w.un, w.ecur);
+#pragma unroll
+    for (int u = 0; u < G::QS; ++u) {
+      const int i = rows[u];
       float2 V[8];
       if constexpr (KC != 0) {
         constexpr uint32_t rb = KC == ROW_PIVOT ? 2u * D : (uint32_t)(D * KC / 8);
         row_values<KC == ROW_PIVOT ? 16 : KC, false, true>(rec + 2u * D + (uint32_t)i * rb, cc, V);
       } else {
         const uint8_t* row = rec + min((uint32_t)roff[i], hd->bytes);
-        switch (code) {
+        switch (rcode[i]) {
           case 8: row_values<8, false, false>(row, cc, V); break;
           case 6: row_values<6, false, false>(row, cc, V); break;
           case 4: row_values<4, false, false>(row, cc, V); break;
@@ -486,35 +622,9 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
           default: row_values<16, false, false>(row, cc, V); break;
         }
       }
-      const double D0 = w.d0[i];
-      const double Mi = (double)w.m[i];
-      const double ki = (double)sk[i];
-      // four columns at a time: j = 16 cc + 4 c4 + e
+      const float2 av = f2(w.af[i]);
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const int j0 = 16 * cc + 4 * c4;
-        const float vv[4] = {V[2 * c4].x, V[2 * c4].y, V[2 * c4 + 1].x, V[2 * c4 + 1].y};
-        double x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          x[e] = __dmul_rn(D0, __dmul_rn(__dmul_rn((double)vv[e], Mi), (double)scol[j0 + e]));
-#pragma unroll 1
-        for (int tau = 0; tau < n; ++tau) {
-          const double ekv = w.ek[tau * D + i];
-          const float4 uu = *reinterpret_cast<const float4*>(ub + tau * D + j0);
-          x[0] = __dadd_rn(x[0], __dmul_rn(ekv, (double)uu.x));
-          x[1] = __dadd_rn(x[1], __dmul_rn(ekv, (double)uu.y));
-          x[2] = __dadd_rn(x[2], __dmul_rn(ekv, (double)uu.z));
-          x[3] = __dadd_rn(x[3], __dmul_rn(ekv, (double)uu.w));
-        }
-        float t[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          t[e] = __double2float_rn(
-              __dmul_rn(__dadd_rn(x[e], __dmul_rn(ki, (double)w.un[j0 + e])), (double)sicol[j0 + e]));
-        T[u][2 * c4] = make_float2(t[0], t[1]);
-        T[u][2 * c4 + 1] = make_float2(t[2], t[3]);
-      }
+      for (int p = 0; p < 8; ++p) T[u][p] = __ffma2_rn(V[p], av, T[u][p]);
     }
     st |= prequant<D, KC, DIRECT>(rec, roff, rcode, rperm, phi, hd->bytes, grp, rg, cc, T);
   }
@@ -523,7 +633,7 @@ __device__ __forceinline__ uint32_t wtile(const WindowArgs& a, const WLay& L, co
 }
 
 template <int D>
-__global__ void __launch_bounds__(WGeo<D>::NT, 2) k_window_step(const WindowArgs a) {
+__global__ void __launch_bounds__(WGeo<D>::NT, 3) k_window_step(const WindowArgs a) {
   using G = PGeo<D>;
   constexpr int NC = WGeo<D>::NC;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -562,7 +672,7 @@ __global__ void __launch_bounds__(WGeo<D>::NT, 2) k_window_step(const WindowArgs
         // loads for the tiles after this one: issued now, used later
         const int nnxt = wcount(a, nxt);
         const WScal nn = wscal(a, blockIdx.x + (it + 2) * gridDim.x);
-        if (it >= 2 && !mbar_wait_bounded(&empty[s], (uint32_t)((it >> 1) - 1) & 1u, a.wait_ns)) break;
+        if (it >= 2 && !wait_suspend(&empty[s], (uint32_t)((it >> 1) - 1) & 1u, a.wait_ns)) break;
         if (cur.m >= n_tiles) {
           reinterpret_cast<WHdr*>(stg)->tile = -1;
           mbar_arrive(&full[s]);
@@ -588,22 +698,26 @@ __global__ void __launch_bounds__(WGeo<D>::NT, 2) k_window_step(const WindowArgs
     const int rg = warp * G::RPW + lane / G::LPR;
     WWork w;
     w.redp = reinterpret_cast<double*>(smem + L.redp);
-    w.redo = reinterpret_cast<float*>(smem + L.redo);
+    w.redo = reinterpret_cast<double*>(smem + L.redo);
     w.ek = reinterpret_cast<double*>(smem + L.ek);
     w.a = reinterpret_cast<double*>(smem + L.a);
+    w.b = reinterpret_cast<double*>(smem + L.b);
+    w.kd = reinterpret_cast<double*>(smem + L.kd);
+    w.qd = reinterpret_cast<double*>(smem + L.qd);
     w.d0 = reinterpret_cast<double*>(smem + L.d0);
-    w.b = reinterpret_cast<float*>(smem + L.b);
     w.m = reinterpret_cast<float*>(smem + L.m);
     w.un = reinterpret_cast<float*>(smem + L.un);
+    w.af = reinterpret_cast<float*>(smem + L.af);
+    w.ecur = reinterpret_cast<float*>(smem + L.ecur);
     w.ag = reinterpret_cast<double*>(smem + L.ag);
     uint32_t st = 0;
     for (int it = 0;; ++it) {
       const int s = it & 1;
-      const uint8_t* stg = smem + (size_t)s * L.stage;
+      uint8_t* stg = smem + (size_t)s * L.stage;
       const WHdr* hd = reinterpret_cast<const WHdr*>(stg);
       // a thread that gives up records the iteration, so that every consumer
       // takes the same decision after the barrier
-      if (!mbar_wait_bounded(&full[s], (uint32_t)(it >> 1) & 1u, a.wait_ns)) abort_sh = it + 1;
+      if (!wait_suspend(&full[s], (uint32_t)(it >> 1) & 1u, a.wait_ns)) abort_sh = it + 1;
       consumer_sync(NC);  // stage s is in for every consumer, or someone gave up
       if (tid == 0 && it > 0) mbar_arrive(&empty[s ^ 1]);  // the previous tile is done
       if (*reinterpret_cast<volatile int*>(&abort_sh) == it + 1) {
