@@ -190,10 +190,15 @@ sq_status sq_decode_step_host(sq_handle* h, void* pool, const float* q, const fl
  *     S_ij = E_-1,i S0_ij + sum_{tau<n} E_tau,i k_tau,i u_tau,j   (S0 the frozen state)
  *     u_j  = fp32(beta (v_j - sum_i S_ij k_i))
  *     o_j  = fp32(sum_i (S_ij + k_i u_j) q_i)
- * in fp64 (u and o rounded once), appends (k, u, G_n) as row n of the
- * buffer, and at n + 1 = W requantizes S + k u^T (formed in fp64, scaled by
- * fp32(1 / c_j), rounded to fp32) in place with the rules of sq_decode_step,
- * then empties the buffer. Inside a window the pool is only read.
+ * in fp64 (u and o rounded once), and appends (k, u, G_n) as row n of the
+ * buffer. At n + 1 = W it forms the state in the record's column-normalised
+ * units in fp32, the way sq_decode_step forms its updated state:
+ *     T_ij = fmaf(V_ij, a_i, t_ij),  t_ij = fmaf(e_tau,i, w_tau,j, t_ij) over
+ *     tau = 0 .. W-1 from t = 0,  a_i = fp32(E_-1,i M_i) (M_i the row scale,
+ *     1 for a pivot row), e_tau,i = fp32(E_tau,i k_tau,i) (E = 1 for the last
+ *     token), w_tau,j = fp32(u_tau,j fp32(1 / c_j)),
+ * requantizes T in place with the rules of sq_decode_step and empties the
+ * buffer. Inside a window the pool is only read.
  *   window_buf device, sq_window_buffer_bytes() bytes, caller-owned; record
  *            of (slot s, value head h) at (s h_v + h) record_bytes:
  *            [int32 count, 12 zero bytes][k: W x d fp32][u: W x d fp32]
