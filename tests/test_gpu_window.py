@@ -22,7 +22,7 @@ import torch
 import oracle
 from quantized_linear_attention_sq_b200 import _abi, synth
 from tests.gpu_util import (THREADS, Stats, compare_slots, gpu_pool_for, oracle_warm_state, slot_bytes, to_dev)
-from tests.helpers import oracle_for, rel_l2
+from tests.helpers import oracle_for, random_calib, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -52,14 +52,18 @@ def compare_windows(ref: np.ndarray, got: np.ndarray, rb: int, W: int, d: int, g
     return bool(diff.any())
 
 
-def run_window_parity(cid: int, W: int, steps: int, check_requests=None, batch=None):
-    w = synth.workload(cid, batch=batch)
+def run_window_parity(cid, W: int, steps: int, check_requests=None, batch=None, slot_perm=None, n_slots=None):
+    """cid: a workload id, or a synth.Workload. slot_perm: [B] GPU pool slot
+    of each request (default: request b in slot b) in a pool of n_slots."""
+    w = cid if isinstance(cid, synth.Workload) else synth.workload(cid, batch=batch)
     c = w.cfg
     B = w.B
     reqs = list(range(B)) if check_requests is None else list(check_requests)
     sel = np.asarray(reqs)
     o_ = oracle_for(oracle, w, n_slots=len(reqs))
-    sp = gpu_pool_for(w, B)
+    slots = np.arange(B, dtype=np.int32) if slot_perm is None else np.asarray(slot_perm, np.int32)
+    n_slots = n_slots or B
+    sp = gpu_pool_for(w, n_slots)
     rb, _ = sp.window_buffer_bytes(W)
     assert rb == o_.window_record_bytes(W)
     gd = c.d if c.gate_kind == _abi.SQ_GATE_KEY_CHANNEL else 1
@@ -70,11 +74,12 @@ def run_window_parity(cid: int, W: int, steps: int, check_requests=None, batch=N
     pool_ref = o_.new_pool()
     o_.quantize(pool_ref, S_ref)
     pool = sp.new_pool()
-    sp.quantize_state(pool, S_all)
+    slots_t = torch.from_numpy(slots).cuda()
+    sp.quantize_state(pool, S_all, slots_t)
     del S_all
     wref = o_.new_window_buffer(W)
     wbuf = sp.new_window_buffer(W)
-    gslots = sel.astype(np.int32)
+    gslots = slots[sel]
     assert np.array_equal(slot_bytes(pool, sp, gslots), pool_ref)
     o_dev = torch.empty((B, c.h_v, c.d), device="cuda")
     stats = Stats()
@@ -83,13 +88,13 @@ def run_window_parity(cid: int, W: int, steps: int, check_requests=None, batch=N
     idx = torch.as_tensor(gslots, device="cuda", dtype=torch.long)
     for t in range(steps):
         q, k, v, beta, g = w.step_inputs(t)
-        sp.window_step(pool, wbuf, W, *to_dev(q, k, v, beta, g), o_dev)
+        sp.window_step(pool, wbuf, W, *to_dev(q, k, v, beta, g), o_dev, slots_t)
         o_ref, st_ref = o_.window_step(pool_ref, wref, W, q[sel], k[sel], v[sel], beta[sel], g[sel],
                                        threads=THREADS)
         st_all |= st_ref
         o_got = o_dev.cpu().numpy()[sel]
         stats.worst_o = max(stats.worst_o, rel_l2(o_got, o_ref))
-        got_w = wbuf.view(B * c.h_v, rb).index_select(0, (idx[:, None] * c.h_v + torch.arange(
+        got_w = wbuf.view(n_slots * c.h_v, rb).index_select(0, (idx[:, None] * c.h_v + torch.arange(
             c.h_v, device="cuda")[None]).reshape(-1)).cpu().numpy().reshape(-1)
         u_diff = compare_windows(wref, got_w, rb, W, c.d, gd, counters)
         got = slot_bytes(pool, sp, gslots)
@@ -99,7 +104,7 @@ def run_window_parity(cid: int, W: int, steps: int, check_requests=None, batch=N
         if u_diff or stats.flips + stats.r_flips != f0:
             pv = pool.view(-1, sp.slot_bytes)
             pv[idx] = torch.from_numpy(pool_ref.reshape(len(reqs), -1)).cuda()
-            wv = wbuf.view(B, -1)
+            wv = wbuf.view(n_slots, -1)
             wv[idx] = torch.from_numpy(wref.reshape(len(reqs), -1)).cuda()
     st_gpu = sp.get_status()
     if len(reqs) == B:
@@ -163,4 +168,42 @@ def test_window_bad_count_and_slot():
         sp.window_step(pool, wbuf, 0, q, k, v, beta, g, o)
     with pytest.raises(_abi.SQError):
         sp.window_step(pool, wbuf, 65, q, k, v, beta, g, o)
+    sp.close()
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("gate_kind", [0, 1])
+def test_window_edge_shapes(d, gate_kind):
+    """Every width {2,4,6,8} and pivots mixed, d in {32, 64, 128}, a ragged
+    batch of 5 requests in permuted slots of a pool of 11; W = 3 over 8
+    tokens (two window ends and a partial window)."""
+    rng = np.random.default_rng(2000 + d + gate_kind)
+    B, h_v, h_k = 5, 6, 3
+    bits, piv, col, phi = random_calib(rng, h_v, d, gate_kind, widths=(2, 4, 6, 8), pivot_p=0.15,
+                                       phi_range=(0.3, 3.0))
+    cfg = synth.Config(98, "window-edge", gate_kind, B, h_v, h_k, d, 8, 64.0, (8,), 8, 0.0, 0.5, 1.0, 0, 0.0)
+    w = synth.Workload(cfg, seed=d)
+    cal = w.calib()
+    cal.unit_bits[...] = bits
+    cal.pivot[...] = piv
+    cal.col_scale[...] = col
+    cal.row_impact[...] = phi
+    stats, cnt = run_window_parity(w, 3, 8, slot_perm=np.array([7, 2, 9, 0, 4], np.int32), n_slots=11)
+    print(stats, cnt)
+    stats.check()
+    assert cnt["u_diff"] <= U_ULP_RATE * cnt["u_entries"] + 2, cnt
+
+
+def test_window_too_long_for_shared_memory_is_rejected():
+    """KDA at d = 128 with W = 64: two stages of buffered rows and gates do
+    not fit in one CTA's shared memory; the call is refused on the host."""
+    w = synth.workload(2, batch=2)
+    c = w.cfg
+    sp = gpu_pool_for(w, 2)
+    pool = sp.new_pool()
+    wbuf = sp.new_window_buffer(64)
+    q, k, v, beta, g = to_dev(*w.step_inputs(0))
+    o = torch.zeros((2, c.h_v, c.d), device="cuda")
+    with pytest.raises(_abi.SQError, match="shared memory"):
+        sp.window_step(pool, wbuf, 64, q, k, v, beta, g, o)
     sp.close()
