@@ -57,11 +57,22 @@ def test_kda_layer_config_subset():
     assert rollout <= gu.ROLLOUT_TOL
 
 
+def test_serving_config_all_tiles_two_steps():
+    """Batch 512 x 32 value heads in the launch configuration of the
+    benchmark, every one of the 16 384 tiles checked against the oracle for
+    two steps (from the oracle's FP32 warm-up of all 512 requests)."""
+    w = synth.workload(3)
+    stats, rollout = gu.run_parity(w, 2)
+    _report("serving all tiles", stats, rollout)
+    stats.check()
+    assert rollout <= gu.ROLLOUT_TOL
+
+
 def test_serving_config_full_size_sampled_requests():
     """Batch 512 x 32 value heads in the launch configuration of the benchmark;
-    the oracle follows 8 sampled requests through all 128 steps."""
+    the oracle follows 16 sampled requests through all 128 steps."""
     w = synth.workload(3)
-    reqs = [0, 37, 101, 200, 255, 318, 444, 511]
+    reqs = [0, 37, 64, 101, 150, 200, 222, 255, 290, 318, 360, 401, 444, 470, 499, 511]
     stats, rollout = gu.run_parity(w, w.cfg.steps, check_requests=reqs, use_gpu_warmup=True)
     _report("serving", stats, rollout)
     stats.check()

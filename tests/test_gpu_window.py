@@ -11,8 +11,8 @@ every token the outputs, the window buffers and the pools are compared:
   straddle an fp32 rounding boundary: at most one fp32 ulp, rarely;
 - pools: identical inside a window (the state is frozen) and, after the
   window's requantization, codes identical up to the step's rare 1-LSB flips
-  (the requantized state is formed in the same order of fp64 operations on
-  both sides, so it differs only where the buffered u did).
+  (both sides form the window-end state with the same fp32 operations in
+  the same order, so it differs only where the buffered u did).
 Where anything differs the GPU continues from the oracle's bytes (teacher
 forcing)."""
 import numpy as np
@@ -113,7 +113,7 @@ def run_window_parity(cid, W: int, steps: int, check_requests=None, batch=None, 
     return stats, counters
 
 
-@pytest.mark.parametrize("cid,W,steps", [(0, 4, 11), (0, 16, 35), (0, 1, 5)])
+@pytest.mark.parametrize("cid,W,steps", [(0, 4, 11), (0, 16, 35), (0, 1, 5), (0, 64, 70)])
 def test_window_plumbing(cid, W, steps):
     stats, cnt = run_window_parity(cid, W, steps)
     print(stats, cnt)
@@ -164,6 +164,11 @@ def test_window_bad_count_and_slot():
     sp.window_step(pool, wbuf, W, q, k, v, beta, g, o, torch.tensor([5], dtype=torch.int32, device="cuda"))
     assert sp.get_status() == _abi.SQ_STATUS_BAD_SLOT
     assert (o == 0).all()
+    # an empty batch is a no-op
+    pool1, w1 = pool.clone(), wbuf.clone()
+    sp.window_step(pool, wbuf, W, q[:0], k[:0], v[:0], beta[:0], g[:0], o[:0])
+    assert sp.get_status() == 0
+    assert torch.equal(pool, pool1) and torch.equal(wbuf, w1)
     with pytest.raises(_abi.SQError):
         sp.window_step(pool, wbuf, 0, q, k, v, beta, g, o)
     with pytest.raises(_abi.SQError):
