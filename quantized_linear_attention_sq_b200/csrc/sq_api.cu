@@ -209,7 +209,7 @@ sq_status plan_kernel(int d, bool packed, uint64_t stage_rec, int sm_smem, int o
   if (by_regs < 1) return fail(SQ_ERR_UNSUPPORTED, "step kernel does not fit on an SM");
   p->nstage = 0;
   if (packed) {
-    const int ns = 2;
+    const int ns = sqk::kPackedStages;
     const size_t smem = (size_t)ns * p->stage_bytes + red;
     if (smem > dyn_max) return fail(SQ_ERR_UNSUPPORTED, "record too large for shared memory");
     p->nstage = ns;

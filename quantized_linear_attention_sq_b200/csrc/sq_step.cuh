@@ -38,6 +38,10 @@
 
 namespace sqk {
 
+// Stages of the packed step (the kernel's mbarrier array has this many
+// entries; the host plans exactly this many).
+constexpr int kPackedStages = 2;
+
 template <int D>
 struct PGeo {
   static constexpr int LPR = D / 16;    // lanes per key row (16 columns each)
@@ -841,7 +845,7 @@ template <int D>
 __global__ void __launch_bounds__(PGeo<D>::NT, 4) k_decode_step_packed(const StepArgs a) {
   using G = PGeo<D>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) uint64_t bars[kPackedStages];
   __shared__ __align__(8) uint64_t free_bar;
   __shared__ __align__(16) float wsh[D];
   __shared__ __align__(16) float msh[D];
