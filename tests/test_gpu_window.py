@@ -42,7 +42,8 @@ def compare_windows(ref: np.ndarray, got: np.ndarray, rb: int, W: int, d: int, g
     assert np.array_equal(R[:, u1:], G[:, u1:]), "buffered gates differ"
     ur = R[:, k1:u1].copy().view(np.float32)
     ug = G[:, k1:u1].copy().view(np.float32)
-    diff = ur != ug
+    assert np.array_equal(np.isnan(ur), np.isnan(ug)), "NaN in one buffer and not the other"
+    diff = (ur != ug) & ~np.isnan(ur)
     counters["u_entries"] += ur.size
     if diff.any():
         a, b = ur[diff].astype(np.float64), ug[diff].astype(np.float64)
@@ -93,7 +94,9 @@ def run_window_parity(cid, W: int, steps: int, check_requests=None, batch=None, 
                                        threads=THREADS)
         st_all |= st_ref
         o_got = o_dev.cpu().numpy()[sel]
-        stats.worst_o = max(stats.worst_o, rel_l2(o_got, o_ref))
+        nan = np.isnan(o_ref)
+        assert np.array_equal(nan, np.isnan(o_got)), "NaN outputs differ"
+        stats.worst_o = max(stats.worst_o, rel_l2(np.where(nan, 0, o_got), np.where(nan, 0, o_ref)))
         got_w = wbuf.view(n_slots * c.h_v, rb).index_select(0, (idx[:, None] * c.h_v + torch.arange(
             c.h_v, device="cuda")[None]).reshape(-1)).cpu().numpy().reshape(-1)
         u_diff = compare_windows(wref, got_w, rb, W, c.d, gd, counters)
@@ -212,3 +215,27 @@ def test_window_too_long_for_shared_memory_is_rejected():
     with pytest.raises(_abi.SQError, match="shared memory"):
         sp.window_step(pool, wbuf, 64, q, k, v, beta, g, o)
     sp.close()
+
+
+class _NaNInput(synth.Workload):
+    """The plumbing workload with one NaN in v (request 0, head 1, column 5)
+    at token 2."""
+
+    def step_inputs(self, step, requests=None):
+        q, k, v, beta, g = super().step_inputs(step, requests)
+        if step == 2:
+            reqs = list(range(self.B)) if requests is None else list(requests)
+            if 0 in reqs:
+                v = v.copy()
+                v[reqs.index(0), 1, 5] = np.nan
+        return q, k, v, beta, g
+
+
+def test_window_nan_input_matches_oracle():
+    """A NaN in v makes that column of u NaN for the rest of the window, o
+    NaN, and at the window's end every row of the head holds a NaN: those
+    rows get scale 0 and code 0 (status NaN), on both sides alike."""
+    w = _NaNInput(synth.CONFIGS[0], seed=0)
+    stats, cnt = run_window_parity(w, 4, 9)
+    print(stats, cnt)
+    stats.check()
