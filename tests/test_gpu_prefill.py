@@ -6,8 +6,12 @@
 2. Against the CPU oracle (the textbook recurrence token by token with an
    extended-precision S^T k, then the oracle's quantization): o per token
    and the final state within 1e-4 relative; codes identical except 1-LSB
-   flips on at most 1e-3 of the entries (the two S^T k sums round
-   differently, so the fp32 states differ in their last bits).
+   flips on at most 5e-5 of the entries. The FP32 format sums S^T k in
+   fp32 in a fixed order on the GPU and exactly in the oracle, so the fp32
+   states differ in their last bits and a code flips where the state sits
+   on a rounding boundary (measured: 0 of 16 384 at d = 64 over 64 tokens,
+   30 of 1.57 M for the GDN layer and 8 of 1.05 M for the KDA layer over
+   32 tokens).
 3. The handoff's edge cases: empty prompt, no S0, ragged and clamped
    lengths, permuted slots, a slot out of range.
 """
@@ -24,7 +28,7 @@ pytestmark = pytest.mark.gpu
 
 STATE_TOL = 1e-4
 O_TOL = 1e-4
-PREFILL_FLIP_RATE = 1e-3
+PREFILL_FLIP_RATE = 5e-5
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -142,6 +146,7 @@ def test_prefill_full_batch_sampled_requests():
         for t in range(L):
             assert rel_l2(o_got[:, t], o_ref[:, t]) <= O_TOL
         entries, flips, worst = _compare_codes(o_, ref_pool, pool.cpu().numpy(), reqs)
+        print(f"\n[prefill full batch] entries={entries} flips={flips} worst={worst}")
         assert worst <= 1 and flips <= PREFILL_FLIP_RATE * entries
     finally:
         pk.close()
@@ -188,6 +193,7 @@ def test_prefill_handoff_edge_cases():
         assert not o_got[0, 2:].any() and not o_got[2].any()
         assert rel_l2(o_got[:, :2], o_ref[:, :2]) <= O_TOL and rel_l2(o_got[1], o_ref[1]) <= O_TOL
         entries, flips, worst = _compare_codes(o_, ref_pool, pool.cpu().numpy(), range(4))
+        print(f"\n[prefill edge] entries={entries} flips={flips} worst={worst}")
         assert worst <= 1 and flips <= PREFILL_FLIP_RATE * entries
     finally:
         pk.close()
