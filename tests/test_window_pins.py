@@ -147,3 +147,22 @@ def test_a_window_of_16_drifts_less_than_per_token_requantization(oracle_mod):
     e1 = rel_l2(orc.dequantize(p1)[0], Sf)
     print(f"\nstate error after 128 tokens: window 16 {e16:.4f}, every token {e1:.4f}")
     assert e16 < e1
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+@pytest.mark.parametrize("gate_kind", [0, 1])
+@pytest.mark.parametrize("W", [1, 3, 16, 64])
+def test_window_record_layout(oracle_mod, d, gate_kind, W):
+    """The window record is [int32 count, 12 zero bytes][k: W d fp32]
+    [u: W d fp32][gates: W gd fp32, padded to a multiple of 4 floats]
+    (gd = d per key channel, 1 per head); its size is a multiple of 16 bytes
+    so that its rows can move by bulk copies; the buffer starts empty."""
+    rng = np.random.default_rng(7)
+    bits, piv, col, phi = random_calib(rng, 2, d, gate_kind, widths=(8,), pivot_p=0.0)
+    orc = oracle_mod.Oracle(3, 2, 1, d, gate_kind, bits, piv, col, phi)
+    gd = d if gate_kind else 1
+    expect = 16 + 4 * (2 * W * d + (W * gd + 3) // 4 * 4)
+    assert orc.window_record_bytes(W) == expect
+    assert expect % 16 == 0
+    buf = orc.new_window_buffer(W)
+    assert buf.size == 3 * 2 * expect and not buf.any()
