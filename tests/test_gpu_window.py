@@ -116,7 +116,7 @@ def run_window_parity(cid, W: int, steps: int, check_requests=None, batch=None, 
     return stats, counters
 
 
-@pytest.mark.parametrize("cid,W,steps", [(0, 4, 11), (0, 16, 35), (0, 1, 5), (0, 64, 70)])
+@pytest.mark.parametrize("cid,W,steps", [(0, 4, 11), (0, 16, 35), (0, 1, 5), (0, 64, 70), (0, 16, 200)])
 def test_window_plumbing(cid, W, steps):
     stats, cnt = run_window_parity(cid, W, steps)
     print(stats, cnt)
