@@ -274,7 +274,8 @@ def run_ours(args, rank, world, local_rank, cid=CONFIG_ID):
                      "frac": achieved / peak, "frac_of_datasheet_8tbs": achieved / DATASHEET_HBM_GBS,
                      "traffic": profiled_traffic() if cid == CONFIG_ID else None,
                      "kernel": f"k_decode_step_packed<{c.d}>", "algorithmic_bytes_per_launch": bytes_launch,
-                     "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
+                     "kernel_ms": kern_ms, "kernel_ms_median": statistics.median(per_ms),
+                     "peak_kind": f"{peak_kind} hbm_gbs (copy)"},
         "state": {"bits_per_value": rep["bits_per_value"], "slot_bytes": rep["slot_bytes"],
                   "clip_fraction": clip,
                   "compression_vs_fp32": 32.0 / rep["bits_per_value"], "status_after_setup": setup_status,
