@@ -16,7 +16,11 @@ rule, the delta-rule invariant, closed forms, Proposition 1 of the method,
 the quantizer error bound, brute force over all codes and all fp16 values,
 and the bit accounting printed for Table D3 of the method's paper;
 tests/test_exact_sum_pins.py ties the exact column sums to a second exact
-computation on columns built to sit next to fp32 rounding boundaries.
+computation on columns built to sit next to fp32 rounding boundaries. The
+per-window variant (``window_step``) is pinned by tests/test_window_pins.py
+(the textbook rule inside a window, half a step at its end, the per-token
+step at W = 1, lower drift at W = 16) and tests/test_window_exact.py (an
+exact-rational reference with explicit IEEE roundings).
 """
 from __future__ import annotations
 
